@@ -1,0 +1,163 @@
+"""2:4 fine-grained structured sparsity: selection, compression, reference GEMMs.
+
+TEST INFRASTRUCTURE (see ``oracle/__init__.py``): imported only by tests,
+``__graft_entry__.smoke()`` and the CPU-baseline legs of ``bench.py``.
+
+Follows "Boost Vision Transformer with GPU-Friendly Sparsity and
+Quantization", Abstract: the dense weight matrix is pruned into the 2:4
+structured pattern (in every group of 4 consecutive weights along the
+reduction dimension K, 2 are kept) to use the GPU's 2:4 sparse tensor cores,
+first in fp16 and then, after quantisation, with integer tensors.
+
+Readings where the abstract is silent:
+
+* selection criterion: magnitude.  In each group the two weights of largest
+  |w| are kept; equal magnitudes are broken by position, the lower index
+  winning.  |w| is compared exactly: for fp16/bf16 through the bit pattern
+  with the sign cleared (monotone in |w| for finite values), for int8 as
+  |q|.  Exactly two slots are kept per group even if they hold zeros.
+* storage: values ``Wv[n, 2g+s] = W[n, 4g + i_s]`` (i0 < i1) and one 4-bit
+  code per group, ``i0 | i1 << 2``; two groups per byte, group 2b in the low
+  nibble of ``meta[n, b]``, group 2b+1 in the high nibble.
+* pruned positions hold +0 (bit pattern 0).
+
+Layouts: W [N, K] row-major (K contiguous), X [M, K], Y [M, N].  fp16 arrays
+are numpy float16; bf16 arrays are uint16 bit patterns; int8 arrays int8.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+DTYPES = ("f16", "bf16", "s8")
+
+
+def magnitude(W: np.ndarray, dtype: str) -> np.ndarray:
+    """|w| as an integer whose order equals the order of |w| (finite inputs)."""
+    if dtype == "f16":
+        return (np.ascontiguousarray(W).view(np.uint16) & np.uint16(0x7FFF)).astype(np.int32)
+    if dtype == "bf16":
+        return (np.asarray(W, dtype=np.uint16) & np.uint16(0x7FFF)).astype(np.int32)
+    if dtype == "s8":
+        return np.abs(np.asarray(W, dtype=np.int8).astype(np.int32))
+    raise ValueError(dtype)
+
+
+def select_24(W: np.ndarray, dtype: str) -> np.ndarray:
+    """Kept positions of every group of 4: int array [N, K/4, 2], ascending.
+
+    A stable sort of the group by decreasing magnitude lists equal
+    magnitudes in index order; its first two entries are the kept ones.
+    """
+    N, K = W.shape
+    if K % 4:
+        raise ValueError("K must be a multiple of 4")
+    mag = magnitude(W, dtype).reshape(N, K // 4, 4)
+    order = np.argsort(-mag, axis=-1, kind="stable")
+    return np.sort(order[..., :2], axis=-1)
+
+
+def _zeros_like(W: np.ndarray) -> np.ndarray:
+    return np.zeros(W.shape, dtype=W.dtype)
+
+
+def prune_24(W: np.ndarray, dtype: str) -> np.ndarray:
+    """Masked weight Wm: kept values in place, +0 elsewhere (same dtype)."""
+    N, K = W.shape
+    keep = select_24(W, dtype)
+    Wm = _zeros_like(W)
+    g = np.arange(K // 4)[None, :]
+    rows = np.arange(N)[:, None]
+    for s in range(2):
+        cols = 4 * g + keep[..., s]
+        Wm[rows, cols] = W[rows, cols]
+    return Wm
+
+
+def compress_24(W: np.ndarray, dtype: str):
+    """(Wv [N, K/2], meta [N, K/8] uint8) of the 2:4 selection of W."""
+    N, K = W.shape
+    if K % 8:
+        raise ValueError("K must be a multiple of 8")
+    keep = select_24(W, dtype)
+    g = np.arange(K // 4)[None, :]
+    rows = np.arange(N)[:, None]
+    Wv = np.empty((N, K // 2), dtype=W.dtype)
+    Wv[:, 0::2] = W[rows, 4 * g + keep[..., 0]]
+    Wv[:, 1::2] = W[rows, 4 * g + keep[..., 1]]
+    nib = (keep[..., 0] | (keep[..., 1] << 2)).astype(np.uint8)
+    meta = (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+    return Wv, meta
+
+
+def decompress_24(Wv: np.ndarray, meta: np.ndarray) -> np.ndarray:
+    """Inverse of ``compress_24``: the masked [N, K] weight."""
+    N, Kh = Wv.shape
+    K = 2 * Kh
+    meta = np.asarray(meta, dtype=np.uint8)
+    nib = np.empty((N, K // 4), dtype=np.int64)
+    nib[:, 0::2] = meta & 0xF
+    nib[:, 1::2] = meta >> 4
+    i0 = nib & 3
+    i1 = nib >> 2
+    Wm = np.zeros((N, K), dtype=Wv.dtype)
+    g = np.arange(K // 4)[None, :]
+    rows = np.arange(N)[:, None]
+    Wm[rows, 4 * g + i0] = Wv[:, 0::2]
+    Wm[rows, 4 * g + i1] = Wv[:, 1::2]
+    return Wm
+
+
+def to_f64(A: np.ndarray, dtype: str) -> np.ndarray:
+    """Exact fp64 value of every element."""
+    if dtype == "f16":
+        return np.asarray(A, dtype=np.float16).astype(np.float64)
+    if dtype == "bf16":
+        b = np.asarray(A, dtype=np.uint16).astype(np.uint32) << np.uint32(16)
+        return b.view(np.float32).astype(np.float64)
+    if dtype == "s8":
+        return np.asarray(A, dtype=np.int8).astype(np.float64)
+    raise ValueError(dtype)
+
+
+def gemm_24_ref(X, Wv, meta, bias, dtype: str, rows=None) -> np.ndarray:
+    """fp16/bf16 2:4 layer in fp64: Y = X . decompress(Wv, meta)^T (+ bias[n]).
+
+    ``rows`` selects a subset of X's rows (the result has one row per entry).
+    """
+    Xs = X if rows is None else X[rows]
+    Wm = to_f64(decompress_24(Wv, meta), dtype)
+    Y = to_f64(Xs, dtype) @ Wm.T
+    if bias is not None:
+        Y = Y + to_f64(bias, dtype)[None, :]
+    return Y
+
+
+def gemm_24_s8_ref(X, Wv, meta, rows=None) -> np.ndarray:
+    """Exact int8 2:4 accumulator acc[m, n] = sum_k x[m,k] * wm[n,k] (int64).
+
+    Computed with an fp64 matrix product, which is exact here: every product
+    is an integer of magnitude <= 127*127 and every partial sum is an integer
+    of magnitude <= K*127*127 < 2**53 (asserted), so no rounding occurs in
+    any summation order.
+    """
+    Xs = X if rows is None else X[rows]
+    K = Xs.shape[1]
+    if K * 128 * 128 >= 2 ** 53:
+        raise ValueError("K too large for an exact fp64 accumulation")
+    Wm = decompress_24(Wv, meta).astype(np.float64)
+    acc = Xs.astype(np.float64) @ Wm.T
+    return np.rint(acc).astype(np.int64)
+
+
+def dequant_s8(acc: np.ndarray, scale: np.ndarray, bias=None) -> np.ndarray:
+    """int8 epilogue: y = fp16_rn( fp32(acc) *rn scale[n] [ +rn fp32(bias[n]) ] ).
+
+    One fp32 multiply, then (if bias is given) one fp32 add, each rounded to
+    nearest even, then one round-to-nearest-even to fp16.  fp32(acc) is exact
+    for |acc| < 2**24 and otherwise rounded to nearest even.
+    """
+    v = np.asarray(acc).astype(np.float32)
+    v = (v * np.asarray(scale, dtype=np.float32)[None, :]).astype(np.float32)
+    if bias is not None:
+        v = (v + np.asarray(bias, dtype=np.float16).astype(np.float32)[None, :]).astype(np.float32)
+    return v.astype(np.float16)

@@ -1,0 +1,225 @@
+"""Counter-based seeded generator for the synthetic workloads.
+
+Every random tensor is a named stream of splitmix64 outputs.  Value ``i``
+(``i = 0, 1, ...``) of the stream with key ``k`` is ``mix(k + (i+1)*gamma)``,
+which is exactly the i-th output of Vigna's splitmix64 started at state ``k``
+(gamma = 0x9E3779B97F4A7C15, mix = the published splitmix64 finaliser).  The
+key of a stream is the 64-bit FNV-1a hash of ``"<seed>:<name>"``.
+
+Derived distributions:
+
+* uniform in [0, 1): ``(u64 >> 11) * 2**-53``;
+* normal: Box-Muller on consecutive pairs ``(u1, u2)``:
+  ``r = sqrt(-2 ln(1 - u1))``, values ``r cos(2 pi u2)``, ``r sin(2 pi u2)``,
+  computed in double, scaled by the standard deviation, rounded to fp32
+  (round-to-nearest-even), then to fp16 or bf16 (round-to-nearest-even);
+* uniform integers in [-127, 127]: ``floor(u * 255) - 127``.
+
+The workload recipe (shapes, distributions, the symmetric per-row int8
+quantisation of the int8 weights, the per-tile densities of the tile-wise
+layers) follows the five synthetic configurations of the pruned-weight linear
+layer studied on the GPUSQ-ViT abstract and the Tile-Wise Sparsity slides.
+Nothing here prunes, selects, reorganises or multiplies: that is the method,
+implemented separately by the CUDA library and by the CPU oracle.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, Optional
+
+import numpy as np
+
+GAMMA = np.uint64(0x9E3779B97F4A7C15)
+_M1 = np.uint64(0xBF58476D1CE4E5B9)
+_M2 = np.uint64(0x94D049BB133111EB)
+_CHUNK = 1 << 22
+
+
+def fnv1a64(text: str) -> int:
+    """64-bit FNV-1a hash of the UTF-8 bytes of ``text``."""
+    h = 0xCBF29CE484222325
+    for b in text.encode("utf-8"):
+        h ^= b
+        h = (h * 0x100000001B3) & 0xFFFFFFFFFFFFFFFF
+    return h
+
+
+def _mix(z: np.ndarray) -> np.ndarray:
+    with np.errstate(over="ignore"):
+        z = (z ^ (z >> np.uint64(30))) * _M1
+        z = (z ^ (z >> np.uint64(27))) * _M2
+    return z ^ (z >> np.uint64(31))
+
+
+def splitmix64_stream(key: int, n: int, start: int = 0) -> np.ndarray:
+    """Outputs ``start .. start+n-1`` of the splitmix64 sequence seeded with ``key``."""
+    i = np.arange(start + 1, start + n + 1, dtype=np.uint64)
+    with np.errstate(over="ignore"):
+        return _mix(np.uint64(key) + i * GAMMA)
+
+
+def _stream_key(seed: int, name: str) -> int:
+    return fnv1a64(f"{seed}:{name}")
+
+
+def uniform01(seed: int, name: str, n: int) -> np.ndarray:
+    """``n`` doubles uniform in [0, 1) from stream ``name``."""
+    key = _stream_key(seed, name)
+    out = np.empty(n, dtype=np.float64)
+    for s in range(0, n, _CHUNK):
+        e = min(n, s + _CHUNK)
+        u = splitmix64_stream(key, e - s, s)
+        out[s:e] = (u >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
+    return out
+
+
+def normal(seed: int, name: str, n: int, std: float) -> np.ndarray:
+    """``n`` fp32 values ~ N(0, std^2) (Box-Muller in double, then RNE to fp32)."""
+    key = _stream_key(seed, name)
+    out = np.empty(n, dtype=np.float32)
+    pairs = (n + 1) // 2
+    step = _CHUNK // 2
+    for p0 in range(0, pairs, step):
+        p1 = min(pairs, p0 + step)
+        u = splitmix64_stream(key, 2 * (p1 - p0), 2 * p0)
+        u = (u >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
+        u1, u2 = u[0::2], u[1::2]
+        r = np.sqrt(-2.0 * np.log1p(-u1))
+        th = 2.0 * math.pi * u2
+        z = np.empty(2 * (p1 - p0), dtype=np.float64)
+        z[0::2] = r * np.cos(th)
+        z[1::2] = r * np.sin(th)
+        lo, hi = 2 * p0, min(n, 2 * p1)
+        out[lo:hi] = (z[: hi - lo] * std).astype(np.float32)
+    return out
+
+
+def uniform_int127(seed: int, name: str, n: int) -> np.ndarray:
+    """``n`` int8 values uniform on the integers -127..127."""
+    u = uniform01(seed, name, n)
+    return (np.floor(u * 255.0) - 127.0).astype(np.int8)
+
+
+def f32_to_f16(x: np.ndarray) -> np.ndarray:
+    """fp32 -> fp16, round to nearest even."""
+    return np.asarray(x, dtype=np.float32).astype(np.float16)
+
+
+def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
+    """fp32 -> bf16 bit patterns (uint16), round to nearest even (finite inputs)."""
+    b = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    r = (b + np.uint32(0x7FFF) + ((b >> np.uint32(16)) & np.uint32(1))) >> np.uint32(16)
+    return r.astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns (uint16) -> exact fp32 values."""
+    return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+@dataclass(frozen=True)
+class Config:
+    """One synthetic workload.
+
+    kind: "24_f16" | "24_bf16" | "24_s8" | "tw_f16".
+    layers: list of (name, M, N, K, bias) GEMMs making up one pass.
+    """
+
+    name: str
+    kind: str
+    layers: tuple
+    x_std: float = 1.0
+    w_std: float = 0.02
+    bias_std: float = 0.01
+    G: int = 0
+    col_prune_frac: float = 0.0
+    density_lo: float = 0.0
+    density_hi: float = 0.0
+    shared_w: Optional[str] = None
+    note: str = ""
+
+
+CONFIGS: Dict[str, Config] = {
+    "tiny_f16": Config(
+        "tiny_f16", "24_f16", (("tiny", 64, 256, 256, False),),
+        note="2:4 fp16 GEMM tiny: X[64,256]~N(0,1), W[256,256]~N(0,0.02)"),
+    "vitb_mlp_f16": Config(
+        "vitb_mlp_f16", "24_f16",
+        (("fc1", 12608, 3072, 768, True), ("fc2", 12608, 768, 3072, True)),
+        note="2:4 fp16 ViT-Base MLP, M=64x197 tokens, fused bias ~N(0,0.01)"),
+    "vitl_mlp_s8": Config(
+        "vitl_mlp_s8", "24_s8", (("fc1", 6304, 4096, 1024, False),),
+        note="2:4 int8 ViT-Large MLP fc1, M=32x197, per-row symmetric int8 weights"),
+    "tw_bert_f16": Config(
+        "tw_bert_f16", "tw_f16",
+        (("attn_out", 4096, 768, 768, False), ("ffn_in", 4096, 3072, 768, False)),
+        G=128, col_prune_frac=0.10, density_lo=0.15, density_hi=0.40,
+        note="tile-wise fp16 BERT-base shapes, M=32x128, G=128, ~75% sparse"),
+    "bf16_prefill": Config(
+        "bf16_prefill", "24_bf16", (("proj", 8192, 16384, 4096, False),),
+        shared_w="bf16_large",
+        note="2:4 bf16 prefill X[8192,4096] x W[16384,4096]^T"),
+    "bf16_decode": Config(
+        "bf16_decode", "24_bf16", (("proj", 16, 16384, 4096, False),),
+        shared_w="bf16_large",
+        note="2:4 bf16 decode-shaped X[16,4096] x the same W"),
+}
+
+
+def tw_tile_counts(N: int, G: int, frac: float):
+    """(P, Nk, T): pruned columns round-half-even(frac*N), kept columns, tiles of G kept columns."""
+    P = int(np.rint(frac * N))
+    Nk = N - P
+    T = (Nk + G - 1) // G
+    return P, Nk, T
+
+
+def _layer_inputs(cfg: Config, seed: int, lname: str, M: int, N: int, K: int, bias: bool) -> dict:
+    stem = f"{cfg.name}.{lname}"
+    wstem = f"{cfg.shared_w}.{lname}" if cfg.shared_w else stem
+    d: dict = {"M": M, "N": N, "K": K}
+    if cfg.kind == "24_s8":
+        d["X"] = uniform_int127(seed, stem + ".X", M * K).reshape(M, K)
+        w = normal(seed, wstem + ".W", N * K, cfg.w_std).reshape(N, K)
+        s = (np.abs(w).max(axis=1) / np.float32(127.0)).astype(np.float32)
+        s = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+        q = np.clip(np.rint(w / s[:, None]), -127, 127).astype(np.int8)
+        d["W"] = q
+        d["scale"] = s
+        d["bias"] = None
+        return d
+    to = f32_to_bf16_bits if cfg.kind == "24_bf16" else f32_to_f16
+    d["X"] = to(normal(seed, stem + ".X", M * K, cfg.x_std)).reshape(M, K)
+    d["W"] = to(normal(seed, wstem + ".W", N * K, cfg.w_std)).reshape(N, K)
+    d["bias"] = to(normal(seed, stem + ".bias", N, cfg.bias_std)) if bias else None
+    if cfg.kind == "tw_f16":
+        P, Nk, T = tw_tile_counts(N, cfg.G, cfg.col_prune_frac)
+        u = uniform01(seed, stem + ".density", T)
+        dens = cfg.density_lo + (cfg.density_hi - cfg.density_lo) * u
+        kt = np.clip(np.rint(dens * K), 1, K).astype(np.int32)
+        d["G"] = cfg.G
+        d["n_pruned"] = P
+        d["k_per_tile"] = kt
+    return d
+
+
+def make_inputs(name: str, seed: int = 0, layers=None) -> list:
+    """Inputs of every layer of configuration ``name`` (list of dicts, one per layer).
+
+    Arrays: X [M,K], W [N,K] (dense, before pruning), bias [N] or None, and for
+    int8 the per-row weight scale; fp16 arrays are float16, bf16 arrays are
+    uint16 bit patterns, int8 arrays are int8.  For tile-wise layers also
+    ``G``, ``n_pruned`` and ``k_per_tile`` (workload data: the per-tile kept-row
+    counts drawn from the configured density range).
+    """
+    cfg = CONFIGS[name]
+    out = []
+    for (lname, M, N, K, bias) in cfg.layers:
+        if layers is not None and lname not in layers:
+            continue
+        d = _layer_inputs(cfg, seed, lname, M, N, K, bias)
+        d["layer"] = lname
+        d["kind"] = cfg.kind
+        out.append(d)
+    return out
