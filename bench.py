@@ -1,0 +1,455 @@
+#!/usr/bin/env python
+"""Benchmark of the pruned-weight linear layer Y = X.W^T on B200.
+
+``python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]``
+
+One step is one pass of the workload's sparse layers over one batch of
+synthetic inputs already resident in HBM (default workload: the 2:4 fp16
+ViT-Base MLP, fc1 12608x3072x768 and fc2 12608x768x3072, each with its fused
+bias).  Prints ONE JSON line on rank 0.  Under torchrun every rank runs its
+own batch (weak scaling, no collective on the data path); the reported value
+is all ranks' dense-equivalent FLOPs divided by the slowest rank's time.
+
+``--impl reference`` times the CPU oracle (numpy, fp64) on the host cores on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workload import gen  # noqa: E402
+
+METRIC = "sparse GEMM dense-equiv TFLOP/s and % of B200 sparse tensor peak (or HBM GB/s)"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DTYPE_NAME = {"24_f16": "f16", "24_bf16": "bf16", "24_s8": "s8", "tw_f16": "f16"}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def layer_flops(layers):
+    return sum(2.0 * d["M"] * d["N"] * d["K"] for d in layers)
+
+
+def algorithmic_bytes(d, kind):
+    """X read once, compressed W + metadata (+bias/scale) read once, Y written once."""
+    M, N, K = d["M"], d["N"], d["K"]
+    if kind == "24_s8":
+        return M * K + N * K // 2 + N * K // 8 + 4 * N + 2 * M * N
+    b = 2 * N if d.get("bias") is not None else 0
+    return 2 * M * K + 2 * N * K // 2 + N * K // 8 + b + 2 * M * N
+
+
+# ---------------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{os.environ.get('RANK', '0')}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    if int(parts[0]) != self.idx:
+                        continue
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for name, val in zip(names, parts[5:9]):
+                    if val.lower().startswith("active"):
+                        reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids) and ids[local_rank].isdigit():
+            return int(ids[local_rank])
+    return local_rank
+
+
+# ---------------------------------------------------------------------------------------------
+# our implementation (CUDA library through the C ABI)
+
+class Layer24:
+    """Device-resident buffers of one 2:4 layer, with `copies` rotating X/Y sets."""
+
+    def __init__(self, spg, d, kind, copies):
+        import torch
+        self.spg, self.d, self.kind = spg, d, kind
+        dev = torch.device("cuda")
+        if kind == "24_s8":
+            W = torch.from_numpy(d["W"]).to(dev)
+            X = torch.from_numpy(d["X"]).to(dev)
+            self.scale = torch.from_numpy(d["scale"]).to(dev)
+            self.out_dtype = torch.float16
+        else:
+            tdt = torch.bfloat16 if kind == "24_bf16" else torch.float16
+            W = self._t(d["W"], tdt, dev)
+            X = self._t(d["X"], tdt, dev)
+            self.scale = None
+            self.out_dtype = tdt
+        self.bias = self._t(d["bias"], self.out_dtype, dev) if d.get("bias") is not None else None
+        self.Wv, self.meta = spg.sparse_compress_24(W)
+        del W
+        self.X = [X] + [X.clone() for _ in range(copies - 1)]
+        self.Y = [torch.empty((d["M"], d["N"]), dtype=self.out_dtype, device=dev) for _ in range(copies)]
+
+    @staticmethod
+    def _t(a, tdt, dev):
+        import torch
+        if a is None:
+            return None
+        if tdt == torch.bfloat16:
+            return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+    def run(self, i, X=None, Y=None):
+        X = self.X[i] if X is None else X
+        Y = self.Y[i] if Y is None else Y
+        if self.kind == "24_s8":
+            self.spg.spgemm_24_s8(X, self.Wv, self.meta, self.scale, self.bias, Y=Y)
+        else:
+            self.spg.spgemm_24_f16(X, self.Wv, self.meta, self.bias, Y=Y)
+
+
+class LayerTW:
+    def __init__(self, spg, d, copies, x_layout):
+        import torch
+        self.spg, self.d = spg, d
+        dev = torch.device("cuda")
+        W = torch.from_numpy(d["W"]).to(dev)
+        self.desc = spg.tw_reorganize(W, d["G"], d["n_pruned"], list(d["k_per_tile"]))
+        X = torch.from_numpy(d["X"]).to(dev)
+        if x_layout == spg.SPG_X_KM:
+            X = X.t().contiguous()
+        self.x_layout = x_layout
+        self.X = [X] + [X.clone() for _ in range(copies - 1)]
+        self.Y = [torch.empty((d["M"], d["N"]), dtype=torch.float16, device=dev) for _ in range(copies)]
+        ws = spg.tw_workspace_size(d["M"], d["K"], x_layout)
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+
+    def run(self, i, X=None, Y=None):
+        X = self.X[i] if X is None else X
+        Y = self.Y[i] if Y is None else Y
+        self.spg.spgemm_tw_f16(X, self.desc, self.x_layout, Y=Y, workspace=self.ws, M=self.d["M"])
+
+
+def tw_algorithmic(layers_tw):
+    flops = 0.0
+    byts = 0
+    for L in layers_tw:
+        d = L.d
+        kp = [int(k) for k in d["k_per_tile"]]
+        Nk = d["N"] - d["n_pruned"]
+        G = d["G"]
+        gts = [min(G, Nk - t * G) for t in range(len(kp))]
+        flops += 2.0 * d["M"] * sum(g * k for g, k in zip(gts, kp))
+        byts += 2 * d["M"] * d["K"] + 2 * d["M"] * d["N"] + 2 * sum(g * k for g, k in zip(gts, kp))
+    return flops, byts
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import structured_sparse_gemm_02_b200 as spg
+    spg.lib()
+    torch.cuda.set_device(local_rank)
+    cfg = gen.CONFIGS[args.workload]
+    inputs = gen.make_inputs(args.workload)
+    copies = args.copies
+    kind = cfg.kind
+    if kind == "tw_f16":
+        layers = [LayerTW(spg, d, copies, spg.SPG_X_KM if args.x_km else spg.SPG_X_MK) for d in inputs]
+        flops_alg, bytes_alg = tw_algorithmic(layers)
+    else:
+        layers = [Layer24(spg, d, kind, copies) for d in inputs]
+        flops_alg = layer_flops(inputs) / 2.0
+        bytes_alg = sum(algorithmic_bytes(d, kind) for d in inputs)
+    flops_dense = layer_flops(inputs)
+    stream = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+
+    def step(i):
+        for L in layers:
+            L.run(i % copies)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    if spg.check_device_error() != 0:
+        raise RuntimeError("device error word set during warm-up")
+
+    nl = len(layers)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps * nl + 1)]
+    sampler = ClockSampler(physical_gpu_index(local_rank))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    evs[0].record(stream)
+    e = 1
+    for i in range(args.steps):
+        for L in layers:
+            L.run(i % copies)
+            evs[e].record(stream)
+            e += 1
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    total_ms = evs[0].elapsed_time(evs[-1])
+    per_layer = [[] for _ in range(nl)]
+    for i in range(args.steps):
+        for j in range(nl):
+            k = i * nl + j
+            per_layer[j].append(evs[k].elapsed_time(evs[k + 1]))
+    if spg.check_device_error() != 0:
+        raise RuntimeError("device error word set during the timed region")
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * flops_dense * args.steps / (total_ms * 1e-3) / 1e12
+
+    # end to end through the same public calls with pinned host buffers
+    e2e = measure_e2e(spg, layers, kind, args, stream)
+
+    peaks, src = load_peaks()
+    lay_ms = [float(np.mean(p)) for p in per_layer]
+    if kind == "24_bf16" and inputs[0]["M"] <= 64 or kind == "tw_f16":
+        # HBM-bound shapes: algorithmic bytes per launch over the measured copy bandwidth
+        per_launch_bytes = bytes_alg / nl
+        achieved = per_launch_bytes / (np.mean(lay_ms) * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": src,
+                "kernel": "spgemm24_kernel" if kind != "tw_f16" else "tw_gemm_kernel"}
+    else:
+        # dense-equivalent FLOPs per launch against the 2:4 sparse tensor peak of the dtype:
+        # measured dense bf16 (same rate as fp16) x2 for 2:4 sparsity, x2 again for int8
+        ratio = 2.0 * (2.0 if kind == "24_s8" else 1.0)
+        peak = peaks["bf16_tflops"] * ratio
+        per_launch = flops_dense / nl
+        achieved = per_launch / (np.mean(lay_ms) * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None, "peak_source": f"{src} bf16 dense x{ratio:g}",
+                "kernel": "spgemm24_kernel"}
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": DTYPE_NAME[kind], "data": "synthetic (seeded splitmix64, seed 0)",
+        "config": {"workload": f"{args.workload}: {cfg.note}",
+                   "layers": [f"{d['layer']} {d['M']}x{d['N']}x{d['K']}" for d in inputs],
+                   "l2": f"inputs larger than L2: {copies} rotating X/Y buffer sets",
+                   "parallelism": f"dp{world} (each rank its own batch, no collective)"},
+        "effective_tflops": world * flops_alg * args.steps / (total_ms * 1e-3) / 1e12,
+        "per_layer_us": [1e3 * v for v in lay_ms],
+        "roofline": roof,
+        "e2e": e2e,
+        "gpu_launches": args.steps * nl * (2 if (kind == "tw_f16" and not args.x_km) else 1),
+        "clocks": clocks,
+    }
+    return out
+
+
+def measure_e2e(spg, layers, kind, args, stream):
+    import torch
+    steps = max(3, min(args.e2e_steps, args.steps))
+    hx, hy = [], []
+    for L in layers:
+        hx.append(L.X[0].cpu().pin_memory())
+        hy.append(torch.empty(L.Y[0].shape, dtype=L.Y[0].dtype).pin_memory())
+    bi = sum(t.numel() * t.element_size() for t in hx)
+    bo = sum(t.numel() * t.element_size() for t in hy)
+
+    def once():
+        for L, x, y in zip(layers, hx, hy):
+            L.X[0].copy_(x, non_blocking=True)
+            L.run(0)
+            y.copy_(L.Y[0], non_blocking=True)
+
+    once()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        once()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    flops = sum(2.0 * L.d["M"] * L.d["N"] * L.d["K"] for L in layers)
+    return {"value": flops / (ms * 1e-3) / 1e12, "unit": "TFLOP/s", "h2d_bytes_per_step": bi,
+            "d2h_bytes_per_step": bo, "ms_per_step": ms, "steps": steps}
+
+
+# ---------------------------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+
+def oracle_step(inputs, kind, rows_frac=1.0):
+    """Run the oracle over (a row sample of) every layer; returns dense-eq FLOPs computed."""
+    from oracle import sparse24 as s24, tilewise as tw
+    flops = 0.0
+    for d in inputs:
+        rows = None
+        M = d["M"]
+        if rows_frac < 1.0:
+            rows = np.arange(0, M, max(1, int(round(1.0 / rows_frac))))
+            M = len(rows)
+        if kind == "tw_f16":
+            r = tw.tw_reorganize(d["W"], d["G"], d["n_pruned"], d["k_per_tile"])
+            tw.tw_gemm_ref(d["X"], r, rows=rows)
+        elif kind == "24_s8":
+            Wv, meta = s24.compress_24(d["W"], "s8")
+            acc = s24.gemm_24_s8_ref(d["X"], Wv, meta, rows=rows)
+            s24.dequant_s8(acc, d["scale"])
+        else:
+            k = DTYPE_NAME[kind]
+            Wv, meta = s24.compress_24(d["W"], k)
+            s24.gemm_24_ref(d["X"], Wv, meta, d.get("bias"), k, rows=rows)
+        flops += 2.0 * M * d["N"] * d["K"]
+    return flops
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def time_oracle(workload, budget_s):
+    cfg = gen.CONFIGS[workload]
+    inputs = gen.make_inputs(workload)
+    frac = 1.0
+    total = sum(2.0 * d["M"] * d["N"] * d["K"] for d in inputs)
+    if total > 2e11:
+        frac = 2e11 / total
+    t0 = time.perf_counter()
+    flops = oracle_step(inputs, cfg.kind, frac)
+    dt = time.perf_counter() - t0
+    reps = 1
+    while time.perf_counter() - t0 < budget_s and reps < 3:
+        flops += oracle_step(inputs, cfg.kind, frac)
+        reps += 1
+    dt = time.perf_counter() - t0
+    sample = (f"{reps} pass(es) of the oracle over "
+              + ("all rows" if frac >= 1.0 else f"every {int(round(1 / frac))}th row")
+              + f" of every layer of {workload} (fp64 numpy, includes compression)")
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
+            "sample": sample, "seconds": dt}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cfg = gen.CONFIGS[args.workload]
+    cb = time_oracle(args.workload, args.cpu_budget)
+    per_step_ms = None
+    return {
+        "impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded splitmix64, seed 0)",
+        "config": {"workload": f"{args.workload}: {cfg.note}", "parallelism": "host cores of rank 0"},
+        "cpu_baseline": cb,
+        "e2e": {"value": cb["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="vitb_mlp_f16", choices=sorted(gen.CONFIGS))
+    ap.add_argument("--copies", type=int, default=3)
+    ap.add_argument("--x-km", action="store_true", help="tile-wise: activations already [K, M]")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    out = run_ours(args, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = time_oracle(args.workload, args.cpu_budget)
+    if world > 1:
+        import torch
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

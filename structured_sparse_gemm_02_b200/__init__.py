@@ -1,0 +1,218 @@
+"""Python binding of the sm_100a structured-sparse GEMM library (``libspgemm.so``).
+
+Argument marshalling only: every function forwards torch tensors' device
+pointers, sizes and the current CUDA stream to the C entry point of the same
+name declared in ``include/spgemm.h``, and raises ``SpgError`` on a non-OK
+status.  There is no fallback: if the shared library is missing or does not
+load, importing the functions raises.  Build it with
+``python -m structured_sparse_gemm_02_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libspgemm.so")
+
+SPG_F16, SPG_BF16, SPG_S8 = 0, 1, 2
+SPG_OUT_F16, SPG_OUT_S32 = 0, 1
+SPG_X_MK, SPG_X_KM = 0, 1
+
+_STATUS = {
+    0: "SPG_OK", 1: "SPG_ERR_INVALID_ARG", 2: "SPG_ERR_UNSUPPORTED_SHAPE", 3: "SPG_ERR_MISALIGNED",
+    4: "SPG_ERR_UNSUPPORTED_DEVICE", 5: "SPG_ERR_CUDA", 6: "SPG_ERR_TIMEOUT",
+}
+
+# Every exported symbol with its (restype, argtypes).
+_i64, _i32, _p, _sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_size_t
+
+
+class SpgTwSizes(ctypes.Structure):
+    _fields_ = [("N", _i64), ("K", _i64), ("Nk", _i64), ("G", _i32), ("T", _i32),
+                ("offsetk_len", _i64), ("wc_elems", _i64)]
+
+
+class SpgTwDesc(ctypes.Structure):
+    _fields_ = [("N", _i64), ("K", _i64), ("Nk", _i64), ("G", _i32), ("T", _i32),
+                ("offsetk_len", _i64), ("offsetn", _p), ("tile_n0", _p), ("tile_kofs", _p),
+                ("k_per_tile", _p), ("offsetk", _p), ("Wc", _p)]
+
+
+SIGNATURES = {
+    "spg_version": (ctypes.c_int, []),
+    "spg_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "spg_check_device_error": (ctypes.c_int, [_p, ctypes.POINTER(ctypes.c_uint32)]),
+    "sparse_prune_24": (ctypes.c_int, [_p, _i64, _p, _i64, _i64, _i64, ctypes.c_int, _p]),
+    "sparse_compress_24": (ctypes.c_int, [_p, _i64, _p, _p, _i64, _i64, ctypes.c_int, _p]),
+    "spgemm_24_f16": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
+    "spgemm_24_s8": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _p, _i64, ctypes.c_int, _i64, _i64, _i64, _p]),
+    "tw_query_sizes": (ctypes.c_int, [_i64, _i64, _i32, _i64, ctypes.POINTER(_i32), ctypes.POINTER(SpgTwSizes)]),
+    "tw_reorganize": (ctypes.c_int, [_p, _i64, _i64, ctypes.POINTER(_i32), ctypes.POINTER(SpgTwDesc), _p]),
+    "tw_workspace_size": (_sz, [_i64, _i64, ctypes.c_int]),
+    "spgemm_tw_f16": (ctypes.c_int, [_p, _i64, ctypes.c_int, ctypes.POINTER(SpgTwDesc), _p, _i64, _i64, _p,
+                                     _sz, _p]),
+}
+
+_lib = None
+
+
+class SpgError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn} failed: {_STATUS.get(status, status)}")
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded shared library (raises if it was not built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m structured_sparse_gemm_02_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, st: int) -> None:
+    if st != 0:
+        raise SpgError(fn, st)
+
+
+def _stream(stream) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(getattr(s, "cuda_stream", s))
+
+
+def _dtype_code(t) -> int:
+    import torch
+    return {torch.float16: SPG_F16, torch.bfloat16: SPG_BF16, torch.int8: SPG_S8}[t.dtype]
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def version() -> int:
+    return lib().spg_version()
+
+
+def check_device_error(stream=None) -> int:
+    """Synchronise ``stream`` and return the device error bits (0 = none)."""
+    bits = ctypes.c_uint32(0)
+    st = lib().spg_check_device_error(_stream(stream), ctypes.byref(bits))
+    if st not in (0, 6):
+        _check("spg_check_device_error", st)
+    return int(bits.value)
+
+
+def sparse_prune_24(W, Wm=None, stream=None):
+    """2:4 magnitude prune of W [N, K] (row pitch = W.stride(0)); returns Wm."""
+    import torch
+    if Wm is None:
+        Wm = torch.empty_like(W)
+    N, K = W.shape
+    _check("sparse_prune_24", lib().sparse_prune_24(
+        _ptr(W), W.stride(0), _ptr(Wm), Wm.stride(0), N, K, _dtype_code(W), _stream(stream)))
+    return Wm
+
+
+def sparse_compress_24(W, Wv=None, meta=None, stream=None):
+    """2:4 compress W [N, K] into (Wv [N, K/2], meta uint8 [N, K/8])."""
+    import torch
+    N, K = W.shape
+    if Wv is None:
+        Wv = torch.empty((N, K // 2), dtype=W.dtype, device=W.device)
+    if meta is None:
+        meta = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device)
+    _check("sparse_compress_24", lib().sparse_compress_24(
+        _ptr(W), W.stride(0), _ptr(Wv), _ptr(meta), N, K, _dtype_code(W), _stream(stream)))
+    return Wv, meta
+
+
+def spgemm_24_f16(X, Wv, meta, bias=None, Y=None, stream=None):
+    """Y [M, N] = X [M, K] . decompress(Wv, meta)^T (+ bias), fp16 or bf16."""
+    import torch
+    M, K = X.shape
+    N = Wv.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    _check("spgemm_24_f16", lib().spgemm_24_f16(
+        _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(bias), _ptr(Y), Y.stride(0), M, N, K,
+        _dtype_code(X), _stream(stream)))
+    return Y
+
+
+def spgemm_24_s8(X, Wv, meta, scale=None, bias=None, Y=None, out_mode=SPG_OUT_F16, stream=None):
+    """int8 2:4 GEMM; out_mode SPG_OUT_F16 (dequantised fp16) or SPG_OUT_S32 (raw int32)."""
+    import torch
+    M, K = X.shape
+    N = Wv.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.int32 if out_mode == SPG_OUT_S32 else torch.float16,
+                        device=X.device)
+    _check("spgemm_24_s8", lib().spgemm_24_s8(
+        _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(scale), _ptr(bias), _ptr(Y), Y.stride(0),
+        out_mode, M, N, K, _stream(stream)))
+    return Y
+
+
+class TwDesc:
+    """Device buffers of a tile-wise descriptor (see ``spg_tw_desc`` in include/spgemm.h)."""
+
+    def __init__(self, N: int, K: int, G: int, n_pruned: int, k_per_tile: Sequence[int], device="cuda"):
+        import torch
+        kpt = (ctypes.c_int32 * len(k_per_tile))(*[int(v) for v in k_per_tile])
+        sz = SpgTwSizes()
+        _check("tw_query_sizes", lib().tw_query_sizes(N, K, G, n_pruned, kpt, ctypes.byref(sz)))
+        self.sizes = sz
+        self.k_host = kpt
+        self.n_pruned = n_pruned
+        i32 = dict(dtype=torch.int32, device=device)
+        self.offsetn = torch.empty(sz.Nk, **i32)
+        self.tile_n0 = torch.empty(sz.T + 1, **i32)
+        self.tile_kofs = torch.empty(sz.T + 1, **i32)
+        self.k_per_tile = torch.empty(sz.T, **i32)
+        self.offsetk = torch.empty(max(1, sz.offsetk_len), **i32)
+        self.Wc = torch.empty(max(1, sz.wc_elems), dtype=torch.float16, device=device)
+        self.c = SpgTwDesc(sz.N, sz.K, sz.Nk, sz.G, sz.T, sz.offsetk_len, self.offsetn.data_ptr(),
+                           self.tile_n0.data_ptr(), self.tile_kofs.data_ptr(), self.k_per_tile.data_ptr(),
+                           self.offsetk.data_ptr(), self.Wc.data_ptr())
+
+
+def tw_reorganize(W, G: int, n_pruned: int, k_per_tile: Sequence[int], stream=None) -> TwDesc:
+    """Condense a dense fp16 W [N, K] into a tile-wise descriptor."""
+    N, K = W.shape
+    d = TwDesc(N, K, G, n_pruned, k_per_tile, device=W.device)
+    _check("tw_reorganize", lib().tw_reorganize(_ptr(W), W.stride(0), n_pruned, d.k_host, ctypes.byref(d.c),
+                                                _stream(stream)))
+    return d
+
+
+def tw_workspace_size(M: int, K: int, x_layout: int) -> int:
+    return int(lib().tw_workspace_size(M, K, x_layout))
+
+
+def spgemm_tw_f16(X, desc: TwDesc, x_layout=SPG_X_MK, Y=None, workspace=None, M: Optional[int] = None,
+                  stream=None):
+    """Tile-wise GEMM: X [M, K] (SPG_X_MK) or [K, M] (SPG_X_KM) -> Y [M, N] fp16."""
+    import torch
+    if M is None:
+        M = X.shape[0] if x_layout == SPG_X_MK else X.shape[1]
+    N = desc.sizes.N
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    ws = tw_workspace_size(M, desc.sizes.K, x_layout)
+    if workspace is None and ws:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=X.device)
+    _check("spgemm_tw_f16", lib().spgemm_tw_f16(
+        _ptr(X), X.stride(0), x_layout, ctypes.byref(desc.c), _ptr(Y), Y.stride(0), M, _ptr(workspace),
+        ws if workspace is not None else 0, _stream(stream)))
+    return Y

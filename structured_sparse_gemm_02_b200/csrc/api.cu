@@ -1,0 +1,114 @@
+// Library-wide entry points (version, status strings, device error word) and
+// the host helpers declared in host.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "host.cuh"
+#include "spgemm.h"
+
+namespace spg {
+
+__device__ uint32_t g_error_word;
+
+namespace {
+constexpr int kMaxDevices = 64;
+int g_dev_ok[kMaxDevices];           // 0 unknown, 1 ok, -1 unsupported
+uint32_t* g_err_ptr[kMaxDevices];
+std::mutex g_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void load_encode() {
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+}
+}  // namespace
+
+spg_status check_device(int* dev_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPG_ERR_CUDA;
+  if (dev_out) *dev_out = dev;
+  if (dev < 0 || dev >= kMaxDevices) return SPG_ERR_UNSUPPORTED_DEVICE;
+  int st = __atomic_load_n(&g_dev_ok[dev], __ATOMIC_ACQUIRE);
+  if (st == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return SPG_ERR_CUDA;
+    st = (major == 10 && minor == 0) ? 1 : -1;
+    __atomic_store_n(&g_dev_ok[dev], st, __ATOMIC_RELEASE);
+  }
+  return st == 1 ? SPG_OK : SPG_ERR_UNSUPPORTED_DEVICE;
+}
+
+uint32_t* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+bool make_tmap_2d(CUtensorMap* map, const void* base, int esize, uint64_t cols, uint64_t rows,
+                  uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+  std::call_once(g_encode_once, load_encode);
+  if (!g_encode) return false;
+  CUtensorMapDataType dt = esize == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                           : esize == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16
+                                        : CU_TENSOR_MAP_DATA_TYPE_UINT32;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {pitch_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace spg
+
+extern "C" {
+
+int spg_version(void) { return 1 * 10000 + 0 * 100 + 0; }
+
+const char* spg_status_string(spg_status s) {
+  switch (s) {
+    case SPG_OK: return "SPG_OK";
+    case SPG_ERR_INVALID_ARG: return "SPG_ERR_INVALID_ARG";
+    case SPG_ERR_UNSUPPORTED_SHAPE: return "SPG_ERR_UNSUPPORTED_SHAPE";
+    case SPG_ERR_MISALIGNED: return "SPG_ERR_MISALIGNED";
+    case SPG_ERR_UNSUPPORTED_DEVICE: return "SPG_ERR_UNSUPPORTED_DEVICE";
+    case SPG_ERR_CUDA: return "SPG_ERR_CUDA";
+    case SPG_ERR_TIMEOUT: return "SPG_ERR_TIMEOUT";
+  }
+  return "SPG_ERR_UNKNOWN";
+}
+
+spg_status spg_check_device_error(spg_stream_t stream, uint32_t* bits) {
+  if (bits) *bits = 0;
+  spg_status st = spg::check_device();
+  if (st != SPG_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SPG_ERR_CUDA;
+  uint32_t v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, spg::g_error_word, sizeof(v)) != cudaSuccess) return SPG_ERR_CUDA;
+  if (v && cudaMemcpyToSymbol(spg::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SPG_ERR_CUDA;
+  if (bits) *bits = v;
+  return v ? SPG_ERR_TIMEOUT : SPG_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,33 @@
+// Host-side helpers shared by the entry points: device checks, the device
+// error word, tensor-map encoding through the driver entry point, and
+// argument validation shorthands.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "spgemm.h"
+
+namespace spg {
+
+// Current device is compute capability 10.0 (result cached per device).
+spg_status check_device(int* dev_out = nullptr);
+
+// Device address of the library's error word on the current device.
+uint32_t* device_error_word();
+
+// 2-D tiled tensor map over a row-major matrix of `rows` x `cols` elements of
+// `esize` bytes with a row pitch of `pitch_bytes`; the box is box_cols x
+// box_rows.  Returns false if the driver rejects the description.
+bool make_tmap_2d(CUtensorMap* map, const void* base, int esize, uint64_t cols, uint64_t rows,
+                  uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128);
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+inline spg_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? SPG_OK : SPG_ERR_CUDA;
+}
+
+}  // namespace spg

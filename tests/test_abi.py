@@ -1,0 +1,68 @@
+"""The C-ABI library loads and exports every entry point its headers declare (no GPU needed)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\*?([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                             text, flags=re.M):
+            names.add(m.group(1))
+    return names
+
+
+def test_headers_declare_the_entry_points():
+    want = {"sparse_prune_24", "sparse_compress_24", "tw_reorganize", "spgemm_24_f16", "spgemm_24_s8",
+            "spgemm_tw_f16", "tw_query_sizes", "tw_workspace_size", "spg_version", "spg_status_string",
+            "spg_check_device_error"}
+    assert want <= _declared()
+
+
+def test_library_exports_every_declared_symbol():
+    import structured_sparse_gemm_02_b200 as spg
+    L = spg.lib()
+    for name in sorted(_declared()):
+        assert hasattr(L, name), name
+    assert set(spg.SIGNATURES) == _declared()
+
+
+def test_host_only_calls():
+    import structured_sparse_gemm_02_b200 as spg
+    L = spg.lib()
+    assert L.spg_version() == 10000
+    assert L.spg_status_string(6) == b"SPG_ERR_TIMEOUT"
+    sz = spg.SpgTwSizes()
+    kpt = (ctypes.c_int32 * 6)(260, 290, 272, 118, 245, 187)
+    assert L.tw_query_sizes(768, 768, 128, 77, kpt, ctypes.byref(sz)) == 0
+    assert (sz.Nk, sz.T) == (691, 6)
+    assert sz.offsetk_len == sum((k + 63) // 64 * 64 for k in (260, 290, 272, 118, 245, 187))
+    assert sz.wc_elems == sz.offsetk_len * 128
+    assert L.tw_query_sizes(768, 768, 64, 77, kpt, ctypes.byref(sz)) == 2      # G must be 128
+    assert L.tw_query_sizes(768, 768, 128, 768, kpt, ctypes.byref(sz)) == 1    # n_pruned < N
+    assert L.tw_workspace_size(4096, 768, spg.SPG_X_MK) == 4096 * 768 * 2
+    assert L.tw_workspace_size(4096, 768, spg.SPG_X_KM) == 0
+
+
+def test_validation_rejects_before_touching_the_device():
+    """Argument errors are reported on the host, before any device query or launch."""
+    import structured_sparse_gemm_02_b200 as spg
+    L = spg.lib()
+    assert L.spgemm_24_f16(None, 256, None, None, None, None, 256, 64, 256, 256, 0, None) == 1
+    assert L.spgemm_24_f16(16, 100, 16, 16, None, 16, 256, 64, 256, 256, 0, None) == 1   # ldx < K
+    assert L.spgemm_24_f16(16, 256, 16, 16, None, 16, 256, 64, 256, 192, 0, None) == 2   # K % 128
+    assert L.spgemm_24_f16(18, 256, 16, 16, None, 16, 256, 64, 256, 256, 0, None) == 3   # X misaligned
+    assert L.spgemm_24_f16(16, 256, 16, 16, None, 16, 256, 64, 256, 256, 7, None) == 1   # dtype
+    assert L.spgemm_24_s8(16, 256, 16, 16, None, None, 16, 256, 0, 64, 256, 256, None) == 1  # scale needed
+    assert L.spgemm_24_s8(16, 256, 16, 16, None, None, 16, 256, 1, 64, 256, 128, None) == 2  # K % 256
+    assert L.sparse_prune_24(16, 6, 16, 6, 2, 6, 0, None) == 2                               # K % 4
+    assert L.sparse_compress_24(16, 12, 16, 16, 2, 12, 0, None) == 2                         # K % 8
+    assert L.sparse_prune_24(16, 8, 16, 8, 0, 8, 0, None) == 0                               # empty: no-op

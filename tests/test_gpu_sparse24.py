@@ -1,0 +1,202 @@
+"""GPU parity of the 2:4 path (prune, compress, fp16/bf16 and int8 GEMMs) against the CPU oracle.
+
+Integer, byte and index results must be bit-exact; fp16/bf16 GEMM outputs must
+satisfy |y - y_ref| <= 1e-3*sqrt(K) + 1e-2*|y_ref| element-wise.
+"""
+import numpy as np
+import pytest
+
+from oracle import compare, sparse24 as s24
+from workload import gen
+from tests.gpu_util import Guarded, need_gpu, to_dev, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def spg():
+    need_gpu()
+    import structured_sparse_gemm_02_b200 as m
+    m.lib()
+    return m
+
+
+def _raw(a):
+    return np.ascontiguousarray(a).view(np.uint8)
+
+
+WEIGHTS = [("tiny_f16", "f16", None), ("vitb_mlp_f16", "f16", "fc2"), ("vitl_mlp_s8", "s8", None),
+           ("bf16_decode", "bf16", None)]
+
+
+@pytest.mark.parametrize("cfg,kind,layer", WEIGHTS)
+def test_prune_and_compress_bit_exact(spg, cfg, kind, layer):
+    import torch
+    d = gen.make_inputs(cfg, layers=[layer] if layer else None)[0]
+    W = d["W"]
+    if W.shape[0] > 2048:
+        W = W[:2048]
+    Wt = to_dev(W, kind)
+    Wm = spg.sparse_prune_24(Wt)
+    Wv, meta = spg.sparse_compress_24(Wt)
+    torch.cuda.synchronize()
+    assert np.array_equal(_raw(to_host(Wm, kind)), _raw(s24.prune_24(W, kind)))
+    rv, rm = s24.compress_24(W, kind)
+    assert np.array_equal(to_host(meta, "u8"), rm)
+    assert np.array_equal(_raw(to_host(Wv, kind)), _raw(rv))
+    # compress(prune(W)) == compress(W); in-place prune
+    Wv2, meta2 = spg.sparse_compress_24(Wm)
+    assert torch.equal(meta2, meta) and torch.equal(Wv2.view(torch.uint8), Wv.view(torch.uint8))
+    spg.sparse_prune_24(Wt, Wt)
+    assert torch.equal(Wt.view(torch.uint8), Wm.view(torch.uint8))
+    assert spg.check_device_error() == 0
+
+
+def test_prune_ties_int8(spg):
+    import torch
+    rng = np.random.default_rng(0)
+    W = rng.choice(np.array([0, 1, -1, 2, -2, 127, -127], np.int8), size=(37, 1024))
+    Wm = spg.sparse_prune_24(torch.from_numpy(W).cuda())
+    Wv, meta = spg.sparse_compress_24(torch.from_numpy(W).cuda())
+    rv, rm = s24.compress_24(W, "s8")
+    assert np.array_equal(Wm.cpu().numpy(), s24.prune_24(W, "s8"))
+    assert np.array_equal(meta.cpu().numpy(), rm) and np.array_equal(Wv.cpu().numpy(), rv)
+
+
+def _gemm_case(spg, kind, X, W, bias):
+    Xt, Wt = to_dev(X, kind), to_dev(W, kind)
+    Wv, meta = spg.sparse_compress_24(Wt)
+    bt = to_dev(bias, kind) if bias is not None else None
+    M, N = X.shape[0], W.shape[0]
+    import torch
+    ldy = (N + 7) // 8 * 8 + (8 if N % 8 else 0)   # ragged N: a padded, 16-byte multiple pitch
+    out = Guarded((M, ldy), torch.float16 if kind == "f16" else torch.bfloat16)
+    Y = out.t[:, :N]
+    spg.spgemm_24_f16(Xt, Wv, meta, bt, Y=Y)
+    assert spg.check_device_error() == 0
+    assert out.intact()
+    pad = out.t[:, N:].contiguous().view(torch.uint8)
+    assert bool((pad == 0xA5).all().item()), "write outside [M, N]"
+    return to_host(Y.contiguous(), kind)
+
+
+@pytest.mark.parametrize("kind", ["f16", "bf16"])
+def test_identity_input_is_bit_exact(spg, kind):
+    """X = I: every output is a single product w*1 accumulated once -> Y = Wm^T exactly."""
+    K, N = 256, 384
+    d = gen.make_inputs("tiny_f16")[0] if kind == "f16" else gen.make_inputs("bf16_decode")[0]
+    W = d["W"][:N, :K] if kind == "bf16" else np.concatenate([d["W"], d["W"][:128] ], 0)[:N, :K]
+    X = np.eye(K, dtype=np.float32)
+    X = X.astype(np.float16) if kind == "f16" else gen.f32_to_bf16_bits(X)
+    Y = _gemm_case(spg, kind, X, W, None)
+    Wm = s24.prune_24(W, kind)
+    assert np.array_equal(_raw(Y), _raw(np.ascontiguousarray(Wm.T)))
+
+
+def test_one_hot_rows_select_columns(spg):
+    K, N = 512, 256
+    W = gen.make_inputs("tiny_f16")[0]["W"]
+    W = np.tile(W, (1, 2))[:N, :K]
+    rng = np.random.default_rng(4)
+    ks = rng.integers(0, K, 64)
+    X = np.zeros((64, K), np.float16)
+    X[np.arange(64), ks] = 1.0
+    Y = _gemm_case(spg, "f16", X, W, None)
+    Wm = s24.prune_24(W, "f16")
+    assert np.array_equal(_raw(Y), _raw(np.ascontiguousarray(Wm[:, ks].T)))
+
+
+def test_tiny_config_parity(spg):
+    d = gen.make_inputs("tiny_f16")[0]
+    Y = _gemm_case(spg, "f16", d["X"], d["W"], None)
+    Wv, meta = s24.compress_24(d["W"], "f16")
+    ref = s24.gemm_24_ref(d["X"], Wv, meta, None, "f16")
+    rep = compare.check_close(Y, ref, d["K"])
+    assert rep["ok"], rep
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 128, 128), (15, 200, 256), (17, 129, 384), (129, 300, 640),
+                                   (200, 64, 1024), (255, 1000, 128)])
+@pytest.mark.parametrize("kind", ["f16", "bf16"])
+def test_ragged_shapes(spg, kind, M, N, K):
+    rng = np.random.default_rng(M * 7 + N)
+    X = rng.standard_normal((M, K)).astype(np.float32)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    b = (rng.standard_normal(N) * 0.01).astype(np.float32)
+    cv = (lambda a: a.astype(np.float16)) if kind == "f16" else gen.f32_to_bf16_bits
+    X, W, b = cv(X), cv(W), cv(b)
+    Y = _gemm_case(spg, kind, X, W, b)
+    Wv, meta = s24.compress_24(W, kind)
+    ref = s24.gemm_24_ref(X, Wv, meta, b, kind)
+    rep = compare.check_close(s24.to_f64(Y, kind), ref, K)
+    assert rep["ok"], rep
+
+
+@pytest.mark.parametrize("layer", ["fc1", "fc2"])
+def test_vitb_full_size_sampled(spg, layer):
+    d = gen.make_inputs("vitb_mlp_f16", layers=[layer])[0]
+    Y = _gemm_case(spg, "f16", d["X"], d["W"], d["bias"])
+    rows = np.unique(np.concatenate([np.arange(0, d["M"], 97), [d["M"] - 1]]))
+    Wv, meta = s24.compress_24(d["W"], "f16")
+    ref = s24.gemm_24_ref(d["X"], Wv, meta, d["bias"], "f16", rows=rows)
+    rep = compare.check_close(Y[rows].astype(np.float64), ref, d["K"])
+    assert rep["ok"], rep
+
+
+def _s8_case(spg, X, W, scale, bias, out_mode):
+    import torch
+    Xt, Wt = torch.from_numpy(X).cuda(), torch.from_numpy(W).cuda()
+    Wv, meta = spg.sparse_compress_24(Wt)
+    M, N = X.shape[0], W.shape[0]
+    ldy = (N + 7) // 8 * 8 + (8 if N % 8 else 0)
+    out = Guarded((M, ldy), torch.int32 if out_mode == spg.SPG_OUT_S32 else torch.float16)
+    Y = out.t[:, :N]
+    st = torch.from_numpy(scale).cuda() if scale is not None else None
+    bt = torch.from_numpy(bias).cuda() if bias is not None else None
+    spg.spgemm_24_s8(Xt, Wv, meta, st, bt, Y=Y, out_mode=out_mode)
+    assert spg.check_device_error() == 0
+    assert out.intact()
+    pad = out.t[:, N:].contiguous().view(torch.uint8)
+    assert bool((pad == 0xA5).all().item()), "write outside [M, N]"
+    return Y.contiguous().cpu().numpy()
+
+
+def test_int8_identity_and_ragged_s32(spg):
+    rng = np.random.default_rng(11)
+    for (M, N, K) in [(256, 256, 256), (17, 131, 512), (300, 64, 768)]:
+        X = rng.integers(-127, 128, (M, K)).astype(np.int8)
+        if M == K:
+            X = np.eye(K, dtype=np.int8)
+        W = rng.integers(-127, 128, (N, K)).astype(np.int8)
+        Y = _s8_case(spg, X, W, None, None, spg.SPG_OUT_S32)
+        Wv, meta = s24.compress_24(W, "s8")
+        assert np.array_equal(Y.astype(np.int64), s24.gemm_24_s8_ref(X, Wv, meta))
+
+
+def test_vitl_int8_full_bit_exact(spg):
+    d = gen.make_inputs("vitl_mlp_s8")[0]
+    Wv, meta = s24.compress_24(d["W"], "s8")
+    acc = s24.gemm_24_s8_ref(d["X"], Wv, meta)
+    Y32 = _s8_case(spg, d["X"], d["W"], None, None, spg.SPG_OUT_S32)
+    assert np.array_equal(Y32.astype(np.int64), acc)
+    Y16 = _s8_case(spg, d["X"], d["W"], d["scale"], None, spg.SPG_OUT_F16)
+    assert np.array_equal(Y16.view(np.uint16), s24.dequant_s8(acc, d["scale"]).view(np.uint16))
+    rng = np.random.default_rng(2)
+    bias = (rng.standard_normal(d["N"]) * 0.01).astype(np.float16)
+    Y16b = _s8_case(spg, d["X"], d["W"], d["scale"], bias, spg.SPG_OUT_F16)
+    assert np.array_equal(Y16b.view(np.uint16), s24.dequant_s8(acc, d["scale"], bias).view(np.uint16))
+
+
+def test_bf16_decode_and_prefill_sampled(spg):
+    dd = gen.make_inputs("bf16_decode")[0]
+    Wv, meta = s24.compress_24(dd["W"], "bf16")
+    Y = _gemm_case(spg, "bf16", dd["X"], dd["W"], None)
+    ref = s24.gemm_24_ref(dd["X"], Wv, meta, None, "bf16")
+    rep = compare.check_close(s24.to_f64(Y, "bf16"), ref, dd["K"])
+    assert rep["ok"], rep
+    dp = gen.make_inputs("bf16_prefill")[0]
+    Yp = _gemm_case(spg, "bf16", dp["X"], dp["W"], None)
+    rows = np.arange(0, dp["M"], 16)[:512]
+    ref = s24.gemm_24_ref(dp["X"], Wv, meta, None, "bf16", rows=rows)
+    rep = compare.check_close(s24.to_f64(Yp[rows], "bf16"), ref, dp["K"])
+    assert rep["ok"], rep
