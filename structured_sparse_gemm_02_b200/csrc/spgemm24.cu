@@ -37,25 +37,37 @@ namespace gemm24 {
 
 enum OutKind { OUT_F16 = 0, OUT_BF16 = 1, OUT_S32 = 2 };
 
-template <bool kInt8, int BN, int STAGES, int OUT>
+// Pair tile: 256 weight rows (128 per CTA of the cluster pair) x BN rows of X
+// (BN/2 loaded by each CTA).  STAGES is the deepest operand ring that fits.
+template <bool kInt8, int BN, int OUT>
 struct Cfg {
-  static constexpr int BM = 128;                       // weight rows per tile (MMA M)
+  static constexpr int BMC = 128;                      // weight rows per CTA (MMA M = 256 per pair)
+  static constexpr int BNH = BN / 2;                   // X rows loaded by each CTA
   static constexpr int KSTEP = kInt8 ? 256 : 128;      // logical K per pipeline stage
-  static constexpr int A_BYTES = BM * 128;             // 128 B of compressed row per stage
-  static constexpr int B_BYTES = BN * 256;             // 256 B of X row per stage (two 128 B atoms)
+  static constexpr int A_BYTES = BMC * 128;            // 128 B of compressed row per stage
+  static constexpr int B_BYTES = BNH * 256;            // 256 B of X row per stage (two 128 B atoms)
   static constexpr int MSTG_BYTES = kInt8 ? 4096 : 2048;  // canonical metadata of the stage (TMA)
   static constexpr int MCP_BYTES = kInt8 ? 0 : 2048;      // fp16/bf16: metadata in tcgen05.cp order
   static constexpr int MCOLS = kInt8 ? 8 : 4;          // TMEM columns of metadata per stage
   static constexpr int OUT_ES = OUT == OUT_S32 ? 4 : 2;
   static constexpr int EPI_BUF = 32 * 32 * OUT_ES;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + MSTG_BYTES + MCP_BYTES;
+  // full[S], mtma[S], meta_full[S], empty[S], acc_full[2], acc_empty[2], mma_done
+  static constexpr int EPI_WARPS = 8;                  // two per tensor-memory lane quadrant
+  static constexpr int THREADS = 32 * (4 + EPI_WARPS);
+  static constexpr int NCH = BN / 32;                  // 32-column chunks of an accumulator
+  static constexpr int CH_HALF = (NCH + 1) / 2;        // chunks of the first epilogue warp of a quadrant
+  static constexpr int BAR_BYTES_MAX = (4 * 8 + 5) * 8 + 16;
+  static constexpr int FIXED = EPI_WARPS * 2 * EPI_BUF + BAR_BYTES_MAX + 1024;
+  static constexpr int STAGES_FIT = (232448 - FIXED) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_MSTG = OFF_B + STAGES * B_BYTES;
   static constexpr int OFF_MCP = OFF_MSTG + STAGES * MSTG_BYTES;
   static constexpr int OFF_EPI = OFF_MCP + STAGES * MCP_BYTES;
-  static constexpr int OFF_BAR = OFF_EPI + 4 * 2 * EPI_BUF;
-  // tma_full[S], meta_full[S], empty[S], acc_full[2], acc_empty[2], mma_done
-  static constexpr int NUM_BARS = 3 * STAGES + 5;
+  static constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * 2 * EPI_BUF;
+  static constexpr int NUM_BARS = 4 * STAGES + 5;
   static constexpr int SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
   static constexpr uint32_t META_COL = 2 * BN;  // metadata ring after the two accumulators
   static constexpr uint32_t TMEM_NEED = 2 * BN + 2 * MCOLS;
@@ -64,10 +76,14 @@ struct Cfg {
                                         : TMEM_NEED <= 128 ? 128
                                         : TMEM_NEED <= 256 ? 256
                                                            : 512;
-  static constexpr uint32_t TX_BYTES = A_BYTES + B_BYTES + MSTG_BYTES;
-  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256, "BN");
+  // bytes counted on the leader's full barrier per stage: operands of both CTAs
+  // (int8 also its metadata; fp16/bf16 metadata completes on a local barrier)
+  static constexpr uint32_t TX_PAIR = 2u * (A_BYTES + B_BYTES + (kInt8 ? MSTG_BYTES : 0));
+  static_assert(BN % 32 == 0 && BN >= 32 && BN <= 256 && BNH % 8 == 0, "BN");
+  static_assert(STAGES >= 2, "at least two stages");
   static_assert(TMEM_NEED <= 512, "tensor memory budget");
   static_assert(SMEM <= 232448, "shared memory budget");
+  static_assert((B_BYTES % 1024) == 0 && ((BNH * 128) % 1024) == 0, "swizzle atoms stay 1024-aligned");
 };
 
 // ---- metadata arrangement ------------------------------------------------------------
@@ -132,19 +148,69 @@ __device__ __forceinline__ uint32_t convert_out(uint32_t acc, float badd, float 
   }
 }
 
-// CTA b computes tiles b, b + gridDim.x, ... of the ceil(N/128) x ceil(M/BN)
-// tile grid (n fastest, so the CTAs in flight share X tiles through L2).
-template <bool kInt8, bool kBF16, int BN, int STAGES, int OUT>
-__global__ void __launch_bounds__(256, 1)
+// Two accumulator values of one output column (rows k and k+1) -> one packed
+// 32-bit word of two 16-bit outputs (row k in the low half), with the same
+// arithmetic as convert_out: fp32 bias add, then one round to nearest even.
+template <int OUT, bool kInt8>
+__device__ __forceinline__ uint32_t convert_pair16(uint32_t a0, uint32_t a1, float badd, float sc, bool has_bias) {
+  float v0, v1;
+  if constexpr (kInt8) {
+    v0 = __fmul_rn(__int2float_rn(static_cast<int>(a0)), sc);
+    v1 = __fmul_rn(__int2float_rn(static_cast<int>(a1)), sc);
+    if (has_bias) {
+      v0 = __fadd_rn(v0, badd);
+      v1 = __fadd_rn(v1, badd);
+    }
+  } else {
+    v0 = __fadd_rn(__uint_as_float(a0), badd);
+    v1 = __fadd_rn(__uint_as_float(a1), badd);
+  }
+  uint32_t w;
+  if constexpr (OUT == OUT_BF16)
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(v1), "f"(v0));
+  else
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(v1), "f"(v0));
+  return w;
+}
+
+// Stage one 32x32 box of 16-bit outputs ([32 rows m][32 columns n], 64 B
+// rows).  Lane n holds p[j] = (row 2j, row 2j+1) of column n.  Neighbour lanes
+// 2i and 2i+1 swap one half so that the even lane holds row 2j and the odd
+// lane row 2j+1 of the column pair (2i, 2i+1); every word lands in a distinct
+// bank (even lanes: banks i, odd lanes: banks 16+i).
+__device__ __forceinline__ void stage_box16(uint8_t* buf, const uint32_t (&p)[16], int lane) {
+  const bool even = (lane & 1) == 0;
+  uint32_t* o = reinterpret_cast<uint32_t*>(buf) + (lane >> 1) + (even ? 0 : 16);
+#pragma unroll
+  for (int j = 0; j < 16; ++j) {
+    // even lanes give away row 2j+1 (high half), odd lanes row 2j (low half)
+    const uint32_t send = even ? (p[j] >> 16) : (p[j] & 0xFFFFu);
+    const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    const uint32_t w = even ? __byte_perm(p[j], recv, 0x5410) : __byte_perm(recv, p[j], 0x7610);
+    o[j * 32] = w;  // row 2j (even) or 2j+1 (odd): 32 words = 2 rows of 64 B apart per j
+  }
+}
+
+// Cluster pairs: pair p = blockIdx.x / 2 computes tiles p, p + gridDim.x/2, ...
+// of the ceil(N/256) x ceil(M/BN) tile grid (n fastest, so the pairs in
+// flight share X tiles through L2).  CTA rank r of the pair loads weight rows
+// [n0 + 128r, +128) and X rows [m0 + r*BN/2, +BN/2); the leader (rank 0)
+// issues the 256 x BN MMAs, which read both CTAs' shared memory and write
+// each CTA's own tensor memory (its 128 weight rows x BN).
+template <bool kInt8, bool kBF16, int BN, int OUT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     spgemm24_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
                     void* __restrict__ Yp, int64_t ldy, const void* __restrict__ bias,
                     const float* __restrict__ scale, int M, int N, int K, uint32_t* err) {
-  using C = Cfg<kInt8, BN, STAGES, OUT>;
+  using C = Cfg<kInt8, BN, OUT>;
+  constexpr int STAGES = C::STAGES;
+  constexpr int BNH = C::BNH;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* tma_full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
-  uint64_t* meta_full = tma_full + STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* mtma = full + STAGES;
+  uint64_t* meta_full = mtma + STAGES;
   uint64_t* empty = meta_full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
@@ -153,19 +219,23 @@ __global__ void __launch_bounds__(256, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int KB = K / C::KSTEP;
-  const int NT = (N + C::BM - 1) / C::BM;
+  const int NT = (N + 255) / 256;
   const int total = NT * ((M + BN - 1) / BN);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&tma_full[s], 1);
-      mbar_init(&meta_full[s], 1);
+      mbar_init(&full[s], 1);
+      mbar_init(&mtma[s], 1);
+      mbar_init(&meta_full[s], 2);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], 2 * C::EPI_WARPS);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -178,21 +248,27 @@ __global__ void __launch_bounds__(256, 1)
     tma_prefetch_desc(&tmY);
   }
   if (warp == 2) {
-    tmem_alloc(tmem_holder, C::TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish_pair();
   }
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // the leader's barriers as seen from either CTA of the pair
+  const uint32_t full_l = mapa_shared(smem_addr(full), 0);
+  const uint32_t meta_full_l = mapa_shared(smem_addr(meta_full), 0);
+  const uint32_t acc_empty_l = mapa_shared(smem_addr(acc_empty), 0);
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer (both CTAs) ----------------
     if (lane == 0) {
       uint32_t g = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
-        const int n0 = (t % NT) * C::BM, m0 = (t / NT) * BN;
+      for (int t = pair; ok && t < total; t += npairs) {
+        const int n0 = (t % NT) * 256 + 128 * int(rank);
+        const int m0 = (t / NT) * BN + BNH * int(rank);
         for (int kb = 0; kb < KB; ++kb, ++g) {
           const int s = g % STAGES;
           const uint32_t use = g / STAGES;
@@ -203,124 +279,129 @@ __global__ void __launch_bounds__(256, 1)
           uint8_t* a_s = smem + C::OFF_A + s * C::A_BYTES;
           uint8_t* b_s = smem + C::OFF_B + s * C::B_BYTES;
           uint8_t* e_s = smem + C::OFF_MSTG + s * C::MSTG_BYTES;
-          mbar_arrive_expect_tx(&tma_full[s], C::TX_BYTES);
-          tma_load_2d(a_s, &tmA, kb * (C::KSTEP / 2), n0, &tma_full[s]);
-          tma_load_2d(b_s, &tmB, kb * C::KSTEP, m0, &tma_full[s]);
-          tma_load_2d(b_s + BN * 128, &tmB, kb * C::KSTEP + C::KSTEP / 2, m0, &tma_full[s]);
+          const uint32_t fb = full_l + 8u * s;
+          if (leader) mbar_arrive_expect_tx(&full[s], C::TX_PAIR);
+          tma_load_2d_pair(a_s, &tmA, kb * (C::KSTEP / 2), n0, fb);
+          tma_load_2d_pair(b_s, &tmB, kb * C::KSTEP, m0, fb);
+          tma_load_2d_pair(b_s + BNH * 128, &tmB, kb * C::KSTEP + C::KSTEP / 2, m0, fb);
           if constexpr (kInt8) {
-            tma_load_2d(e_s, &tmE, kb * 32, n0, &tma_full[s]);
-            tma_load_2d(e_s + 2048, &tmE, kb * 32 + 16, n0, &tma_full[s]);
+            tma_load_2d_pair(e_s, &tmE, kb * 32, n0, fb);
+            tma_load_2d_pair(e_s + 2048, &tmE, kb * 32 + 16, n0, fb);
           } else {
-            tma_load_2d(e_s, &tmE, kb * 16, n0, &tma_full[s]);
+            mbar_arrive_expect_tx(&mtma[s], C::MSTG_BYTES);
+            tma_load_2d(e_s, &tmE, kb * 16, n0, &mtma[s]);
           }
         }
       }
-      // Let every issued copy land before shared memory can be released.
-      for (uint32_t q = (g > uint32_t(STAGES) ? g - STAGES : 0u); q < g; ++q)
-        tail_wait(&tma_full[q % STAGES], (q / STAGES) & 1, err);
+      // Let every issued copy land before shared memory can be released: the
+      // leader's full barriers count both CTAs' operand bytes, the local
+      // metadata barriers this CTA's metadata.
+      for (uint32_t q = (g > uint32_t(STAGES) ? g - STAGES : 0u); q < g; ++q) {
+        if (leader) tail_wait(&full[q % STAGES], (q / STAGES) & 1, err);
+        if constexpr (!kInt8) tail_wait(&mtma[q % STAGES], (q / STAGES) & 1, err);
+      }
     }
   } else if (warp == 1) {
-    // ------------- metadata arrangement (fp16/bf16 only) -------------
+    // ------------- metadata arrangement (fp16/bf16, both CTAs) -------------
     if constexpr (!kInt8) {
       uint32_t g = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+      for (int t = pair; ok && t < total; t += npairs) {
         for (int kb = 0; kb < KB; ++kb, ++g) {
           const int s = g % STAGES;
-          if (!mbar_wait(&tma_full[s], (g / STAGES) & 1, abort_flag, err, ERR_WAIT_FULL)) {
+          if (!mbar_wait(&mtma[s], (g / STAGES) & 1, abort_flag, err, ERR_WAIT_META)) {
             ok = false;
             break;
           }
           permute_meta_f16(smem + C::OFF_MSTG + s * C::MSTG_BYTES, smem + C::OFF_MCP + s * C::MCP_BYTES, lane);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&meta_full[s]);
+          if (lane == 0) mbar_arrive_cluster(meta_full_l + 8u * s);
         }
       }
     }
   } else if (warp == 2) {
-    // ---------------- MMA issuer ----------------
-    constexpr uint32_t kFmt = kInt8 ? 1u : (kBF16 ? 1u : 0u);
-    constexpr uint32_t kCFmt = kInt8 ? 2u : 1u;
-    uint32_t g = 0;
-    int i = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; ok && t < total; t += gridDim.x, ++i) {
-      const int b = i & 1;
-      if (i >= 2 && !mbar_wait(&acc_empty[b], ((i >> 1) - 1) & 1, abort_flag, err, ERR_WAIT_ACC_FREE)) break;
-      tc_fence_after();
-      const uint32_t acc = tmem + uint32_t(b * BN);
-      for (int kb = 0; kb < KB; ++kb, ++g) {
-        const int s = g % STAGES;
-        const uint32_t ph = (g / STAGES) & 1;
-        if (!mbar_wait(&tma_full[s], ph, abort_flag, err, ERR_WAIT_FULL)) {
-          ok = false;
-          break;
-        }
-        if constexpr (!kInt8) {
-          if (!mbar_wait(&meta_full[s], ph, abort_flag, err, ERR_WAIT_META)) {
+    // ---------------- MMA issuer (leader CTA) ----------------
+    if (leader) {
+      constexpr uint32_t kFmt = kInt8 ? 1u : (kBF16 ? 1u : 0u);
+      constexpr uint32_t kCFmt = kInt8 ? 2u : 1u;
+      uint32_t g = 0;
+      int i = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < total; t += npairs, ++i) {
+        const int b = i & 1;
+        if (i >= 2 && !mbar_wait(&acc_empty[b], ((i >> 1) - 1) & 1, abort_flag, err, ERR_WAIT_ACC_FREE)) break;
+        tc_fence_after();
+        const uint32_t acc = tmem + uint32_t(b * BN);
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % STAGES;
+          const uint32_t ph = (g / STAGES) & 1;
+          if (!mbar_wait(&full[s], ph, abort_flag, err, ERR_WAIT_FULL)) {
             ok = false;
             break;
           }
-        }
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t a_s = smem_addr(smem + C::OFF_A + s * C::A_BYTES);
-          const uint32_t b_s = smem_addr(smem + C::OFF_B + s * C::B_BYTES);
-          const uint32_t ecol = tmem + C::META_COL + (g & 1) * C::MCOLS;
-          if constexpr (kInt8) {
-            const uint32_t e_s = smem_addr(smem + C::OFF_MSTG + s * C::MSTG_BYTES);
-            tc_cp_128x128b(ecol, smem_desc(e_s, 2048, 128, LAYOUT_NONE));
-            tc_cp_128x128b(ecol + 4, smem_desc(e_s + 2048, 2048, 128, LAYOUT_NONE));
-          } else {
-            const uint32_t e_s = smem_addr(smem + C::OFF_MCP + s * C::MCP_BYTES);
-            tc_cp_128x128b(ecol, smem_desc(e_s, 2048, 128, LAYOUT_NONE));
+          if constexpr (!kInt8) {
+            if (!mbar_wait(&meta_full[s], ph, abort_flag, err, ERR_WAIT_META)) {
+              ok = false;
+              break;
+            }
           }
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t a_s = smem_addr(smem + C::OFF_A + s * C::A_BYTES);
+            const uint32_t b_s = smem_addr(smem + C::OFF_B + s * C::B_BYTES);
+            const uint32_t ecol = tmem + C::META_COL + (g & 1) * C::MCOLS;
+            if constexpr (kInt8) {
+              const uint32_t e_s = smem_addr(smem + C::OFF_MSTG + s * C::MSTG_BYTES);
+              tc_cp_128x128b_pair(ecol, smem_desc(e_s, 2048, 128, LAYOUT_NONE));
+              tc_cp_128x128b_pair(ecol + 4, smem_desc(e_s + 2048, 2048, 128, LAYOUT_NONE));
+            } else {
+              const uint32_t e_s = smem_addr(smem + C::OFF_MCP + s * C::MCP_BYTES);
+              tc_cp_128x128b_pair(ecol, smem_desc(e_s, 2048, 128, LAYOUT_NONE));
+            }
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint64_t adesc = smem_desc(a_s + 32 * j, 16, 1024, LAYOUT_SW128);
-            const uint64_t bdesc =
-                smem_desc(b_s + (j >> 1) * (BN * 128) + (j & 1) * 64, 16, 1024, LAYOUT_SW128);
-            const uint32_t e = kInt8 ? ecol + 2 * j : ecol + (j & ~1);
-            const uint32_t sel = kInt8 ? 0u : uint32_t(j & 1);
-            tc_mma_sp<kInt8>(acc, adesc, bdesc, e, instr_desc(kFmt, kCFmt, 128, BN, true, sel),
-                             (kb | j) != 0 ? 1u : 0u);
+            for (int j = 0; j < 4; ++j) {
+              const uint64_t adesc = smem_desc(a_s + 32 * j, 16, 1024, LAYOUT_SW128);
+              const uint64_t bdesc =
+                  smem_desc(b_s + (j >> 1) * (BNH * 128) + (j & 1) * 64, 16, 1024, LAYOUT_SW128);
+              const uint32_t e = kInt8 ? ecol + 2 * j : ecol + (j & ~1);
+              const uint32_t sel = kInt8 ? 0u : uint32_t(j & 1);
+              tc_mma_sp_pair<kInt8>(acc, adesc, bdesc, e, instr_desc(kFmt, kCFmt, 256, BN, true, sel),
+                                    (kb | j) != 0 ? 1u : 0u);
+            }
+            tc_commit_pair(&empty[s], 0x3);
           }
-          tc_commit(&empty[s]);
+          __syncwarp();
         }
+        if (!ok) break;
+        if (lane == 0) tc_commit_pair(&acc_full[b], 0x3);
         __syncwarp();
       }
-      if (!ok) break;
-      if (lane == 0) tc_commit(&acc_full[b]);
+      if (lane == 0) tc_commit_pair(mma_done, 0x3);
       __syncwarp();
     }
-    if (lane == 0) {
-      tc_commit(mma_done);
-      tail_wait(mma_done, 0, err);
-    }
+    // both CTAs: every MMA reading this CTA's shared memory or writing its
+    // tensor memory has completed once the leader's final commit arrives
+    if (lane == 0) tail_wait(mma_done, 0, err);
     __syncwarp();
   } else if (warp >= 4) {
-    // ---------------- epilogue ----------------
-    const int q = warp & 3;  // tensor-memory lane quadrant of this warp
-    uint8_t* epi = smem + C::OFF_EPI + q * 2 * C::EPI_BUF;
+    // ---------------- epilogue (both CTAs) ----------------
+    // Warp w reads tensor-memory lanes 32*(w%4).. (its quadrant) and one half
+    // of the accumulator's 32-column chunks; the next chunk's tcgen05.ld is in
+    // flight while the current one is converted and stored.
+    const int q = warp & 3;
+    const int half = (warp - 4) >> 2;
+    const int c_lo = half ? C::CH_HALF : 0;
+    const int c_hi = half ? C::NCH : C::CH_HALF;
+    uint8_t* epi = smem + C::OFF_EPI + (warp - 4) * 2 * C::EPI_BUF;
     uint32_t cc = 0;  // output boxes staged by this warp so far
     int i = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++i) {
-      const int n0 = (t % NT) * C::BM, m0 = (t / NT) * BN;
+    for (int t = pair; t < total; t += npairs, ++i) {
+      const int n0 = (t % NT) * 256 + 128 * int(rank), m0 = (t / NT) * BN;
       const int b = i & 1;
       if (!mbar_wait(&acc_full[b], (i >> 1) & 1, abort_flag, err, ERR_WAIT_ACC)) break;
       tc_fence_after();
-      uint32_t r[BN / 32][32];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c)
-        tmem_ld_32x32b_x32(tmem + (uint32_t(32 * q) << 16) + uint32_t(b * BN + 32 * c), r[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[b]);
-
       const int nb = n0 + 32 * q;
-      if (nb >= N) continue;
       const int n = nb + lane;
       float badd = 0.f, sc = 0.f;
       bool has_bias = false;
@@ -339,42 +420,77 @@ __global__ void __launch_bounds__(256, 1)
         }
       }
       const bool full_n = nb + 32 <= N;
+      const uint32_t tbase = tmem + (uint32_t(32 * q) << 16) + uint32_t(b * BN);
+      if (c_lo >= c_hi) {  // narrow tiles: this warp has no chunk, only hands the accumulator back
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc_empty_l + 8u * b);
+        continue;
+      }
+      uint32_t r[2][32];
+      tmem_ld_32x32b_x32(tbase + 32 * c_lo, r[0]);
+      tmem_ld_wait(r[0]);
+#pragma unroll 1
+      for (int c = c_lo; c < c_hi; c += 2) {
+        // two chunks per iteration so that register indices stay static
 #pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        const int mb = m0 + 32 * c;
-        if (mb >= M) continue;
-        if (full_n) {
-          if (cc >= 2) {
-            if (lane == 0) bulk_wait_read<1>();
+        for (int u = 0; u < 2; ++u) {
+          const int cu = c + u;
+          if (cu >= c_hi) break;
+          const bool more = cu + 1 < c_hi;
+          if (more) tmem_ld_32x32b_x32(tbase + 32 * (cu + 1), r[u ^ 1]);
+          const int mb = m0 + 32 * cu;
+          if (nb < N && mb < M) {
+            uint32_t (&h)[32] = r[u];
+            if constexpr (C::OUT_ES == 4) {
+#pragma unroll
+              for (int k = 0; k < 32; ++k) h[k] = convert_out<OUT, kInt8>(h[k], badd, sc, has_bias);
+            } else {
+              // packed pairs (rows 2j, 2j+1) kept in h[0..15]
+#pragma unroll
+              for (int j = 0; j < 16; ++j) h[j] = convert_pair16<OUT, kInt8>(h[2 * j], h[2 * j + 1], badd, sc, has_bias);
+            }
+            if (full_n) {
+              if (cc >= 2) {
+                if (lane == 0) bulk_wait_read<1>();
+                __syncwarp();
+              }
+              uint8_t* buf = epi + (cc & 1) * C::EPI_BUF;
+              if constexpr (C::OUT_ES == 4) {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) reinterpret_cast<uint32_t*>(buf)[k * 32 + lane] = h[k];
+              } else {
+                stage_box16(buf, reinterpret_cast<const uint32_t(&)[16]>(h), lane);
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&tmY, buf, nb, mb);
+                bulk_commit();
+              }
+              __syncwarp();
+              ++cc;
+            } else if (n < N) {
+              // ragged right edge: bounds-checked direct stores
+#pragma unroll
+              for (int k = 0; k < 32; ++k) {
+                if (mb + k >= M) continue;
+                if constexpr (C::OUT_ES == 4)
+                  static_cast<uint32_t*>(Yp)[int64_t(mb + k) * ldy + n] = h[k];
+                else
+                  static_cast<uint16_t*>(Yp)[int64_t(mb + k) * ldy + n] =
+                      static_cast<uint16_t>((k & 1) ? (h[k >> 1] >> 16) : (h[k >> 1] & 0xFFFFu));
+              }
+            }
+          }
+          if (more) {
+            tmem_ld_wait(r[u ^ 1]);
+          }
+          if (cu + 1 == c_hi) {
+            // every chunk of this warp is read: hand the accumulator back
+            tc_fence_before();
             __syncwarp();
-          }
-          uint8_t* buf = epi + (cc & 1) * C::EPI_BUF;
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const uint32_t v = convert_out<OUT, kInt8>(r[c][k], badd, sc, has_bias);
-            if constexpr (C::OUT_ES == 4)
-              reinterpret_cast<uint32_t*>(buf)[k * 32 + lane] = v;
-            else
-              reinterpret_cast<uint16_t*>(buf)[k * 32 + lane] = static_cast<uint16_t>(v);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmY, buf, nb, mb);
-            bulk_commit();
-          }
-          __syncwarp();
-          ++cc;
-        } else if (n < N) {
-          // ragged right edge: bounds-checked direct stores
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            if (mb + k >= M) continue;
-            const uint32_t v = convert_out<OUT, kInt8>(r[c][k], badd, sc, has_bias);
-            if constexpr (C::OUT_ES == 4)
-              static_cast<uint32_t*>(Yp)[int64_t(mb + k) * ldy + n] = v;
-            else
-              static_cast<uint16_t*>(Yp)[int64_t(mb + k) * ldy + n] = static_cast<uint16_t>(v);
+            if (lane == 0) mbar_arrive_cluster(acc_empty_l + 8u * b);
           }
         }
       }
@@ -383,11 +499,12 @@ __global__ void __launch_bounds__(256, 1)
     __syncwarp();
   }
 
+  __syncwarp();
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // neither CTA leaves while its peer may still signal or read it
   if (warp == 2) {
     tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
+    tmem_dealloc_pair(tmem, C::TMEM_COLS);
   }
 }
 
@@ -403,27 +520,61 @@ int sm_count() {
   return cached[dev];
 }
 
-template <bool kInt8, bool kBF16, int BN, int STAGES, int OUT>
+// Cluster pairs of `kern` that fit on the device at once (cached per kernel and device).
+int resident_pairs(const void* kern, int smem, int threads) {
+  struct Entry { const void* k; int dev; int n; };
+  static Entry cache[64];
+  static int used = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  for (int i = 0; i < used; ++i)
+    if (cache[i].k == kern && cache[i].dev == dev) return cache[i].n;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads), 1, 1);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    n = sm_count() / 2;
+  }
+  if (used < 64) cache[used++] = Entry{kern, dev, n};
+  return n;
+}
+
+template <bool kInt8, bool kBF16, int BN, int OUT>
 spg_status launch(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,
                   const float* scale, void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
-  using C = Cfg<kInt8, BN, STAGES, OUT>;
+  using C = Cfg<kInt8, BN, OUT>;
   const int es = kInt8 ? 1 : 2;
   CUtensorMap tmA, tmB, tmE, tmY;
   if (!make_tmap_2d(&tmA, Wv, es, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2) * es, 128 / es, 128, true) ||
-      !make_tmap_2d(&tmB, X, es, uint64_t(K), uint64_t(M), uint64_t(ldx) * es, 128 / es, BN, true) ||
+      !make_tmap_2d(&tmB, X, es, uint64_t(K), uint64_t(M), uint64_t(ldx) * es, 128 / es, C::BNH, true) ||
       !make_tmap_2d(&tmE, meta, 1, uint64_t(K / 8), uint64_t(N), uint64_t(K / 8), 16, 128, false) ||
       !make_tmap_2d(&tmY, Y, C::OUT_ES, uint64_t(N), uint64_t(M), uint64_t(ldy) * C::OUT_ES, 32, 32, false))
     return SPG_ERR_CUDA;
   uint32_t* err = device_error_word();
   if (!err) return SPG_ERR_CUDA;
-  auto kern = spgemm24_kernel<kInt8, kBF16, BN, STAGES, OUT>;
+  auto kern = spgemm24_kernel<kInt8, kBF16, BN, OUT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
     return SPG_ERR_CUDA;
-  const int64_t tiles = ((N + C::BM - 1) / C::BM) * ((M + BN - 1) / BN);
-  const int grid = static_cast<int>(tiles < sm_count() ? tiles : sm_count());
-  kern<<<grid, 256, C::SMEM, stream>>>(tmA, tmB, tmE, tmY, Y, ldy, bias, scale, static_cast<int>(M),
-                                       static_cast<int>(N), static_cast<int>(K), err);
+  const int64_t tiles = ((N + 255) / 256) * ((M + BN - 1) / BN);
+  const int64_t pairs_max = resident_pairs(reinterpret_cast<const void*>(kern), C::SMEM, C::THREADS);
+  if (pairs_max <= 0) return SPG_ERR_CUDA;
+  const int pairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
+  kern<<<2 * pairs, C::THREADS, C::SMEM, stream>>>(tmA, tmB, tmE, tmY, Y, ldy, bias, scale, static_cast<int>(M),
+                                            static_cast<int>(N), static_cast<int>(K), err);
   return launch_status();
+}
+
+// X rows per pair tile: small batches take narrow tiles, large ones the widest
+// tile whose two accumulators and metadata ring fit in tensor memory.
+template <bool kInt8, bool kBF16, int OUT>
+spg_status dispatch(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,
+                    const float* scale, void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t s) {
+  if (M <= 32) return launch<kInt8, kBF16, 32, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s);
+  if (M <= 128) return launch<kInt8, kBF16, 128, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s);
+  return launch<kInt8, kBF16, 224, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s);
 }
 
 spg_status validate_common(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, void* Y, int64_t ldy,
@@ -455,9 +606,8 @@ spg_status spgemm_24_f16(const void* X, int64_t ldx, const void* Wv, const uint8
   st = check_device();
   if (st != SPG_OK) return st;
   auto s = reinterpret_cast<cudaStream_t>(stream);
-  if (dtype == SPG_F16)
-    return launch<false, false, 128, 4, OUT_F16>(X, ldx, Wv, meta, bias, nullptr, Y, ldy, M, N, K, s);
-  return launch<false, true, 128, 4, OUT_BF16>(X, ldx, Wv, meta, bias, nullptr, Y, ldy, M, N, K, s);
+  if (dtype == SPG_F16) return dispatch<false, false, OUT_F16>(X, ldx, Wv, meta, bias, nullptr, Y, ldy, M, N, K, s);
+  return dispatch<false, true, OUT_BF16>(X, ldx, Wv, meta, bias, nullptr, Y, ldy, M, N, K, s);
 }
 
 spg_status spgemm_24_s8(const int8_t* X, int64_t ldx, const int8_t* Wv, const uint8_t* meta, const float* scale,
@@ -476,8 +626,8 @@ spg_status spgemm_24_s8(const int8_t* X, int64_t ldx, const int8_t* Wv, const ui
   if (st != SPG_OK) return st;
   auto s = reinterpret_cast<cudaStream_t>(stream);
   if (out_mode == SPG_OUT_S32)
-    return launch<true, false, 128, 3, OUT_S32>(X, ldx, Wv, meta, nullptr, nullptr, Y, ldy, M, N, K, s);
-  return launch<true, false, 128, 4, OUT_F16>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s);
+    return dispatch<true, false, OUT_S32>(X, ldx, Wv, meta, nullptr, nullptr, Y, ldy, M, N, K, s);
+  return dispatch<true, false, OUT_F16>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s);
 }
 
 }  // extern "C"
