@@ -50,15 +50,16 @@ struct Cfg {
   static constexpr int MCP_BYTES = kInt8 ? 0 : 2048;      // fp16/bf16: metadata in tcgen05.cp order
   static constexpr int MCOLS = kInt8 ? 8 : 4;          // TMEM columns of metadata per stage
   static constexpr int OUT_ES = OUT == OUT_S32 ? 4 : 2;
-  static constexpr int EPI_BUF = 32 * 32 * OUT_ES;
+  // staging per epilogue warp: 16-bit outputs double-buffer a 4 KB box per warp
+  // pair (2 KB per warp and buffer); int32 outputs one 4 KB box per warp
+  static constexpr int EPI_BUF = OUT_ES == 2 ? 2 * 2048 : 4096;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + MSTG_BYTES + MCP_BYTES;
   // full[S], mtma[S], meta_full[S], empty[S], acc_full[2], acc_empty[2], mma_done
   static constexpr int EPI_WARPS = 8;                  // two per tensor-memory lane quadrant
   static constexpr int THREADS = 32 * (4 + EPI_WARPS);
   static constexpr int NCH = BN / 32;                  // 32-column chunks of an accumulator
-  static constexpr int CH_HALF = (NCH + 1) / 2;        // chunks of the first epilogue warp of a quadrant
   static constexpr int BAR_BYTES_MAX = (4 * 8 + 5) * 8 + 16;
-  static constexpr int FIXED = EPI_WARPS * 2 * EPI_BUF + BAR_BYTES_MAX + 1024;
+  static constexpr int FIXED = EPI_WARPS * EPI_BUF + BAR_BYTES_MAX + 1024;
   static constexpr int STAGES_FIT = (232448 - FIXED) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int OFF_A = 0;
@@ -66,7 +67,7 @@ struct Cfg {
   static constexpr int OFF_MSTG = OFF_B + STAGES * B_BYTES;
   static constexpr int OFF_MCP = OFF_MSTG + STAGES * MSTG_BYTES;
   static constexpr int OFF_EPI = OFF_MCP + STAGES * MCP_BYTES;
-  static constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * 2 * EPI_BUF;
+  static constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * EPI_BUF;
   static constexpr int NUM_BARS = 4 * STAGES + 5;
   static constexpr int SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
   static constexpr uint32_t META_COL = 2 * BN;  // metadata ring after the two accumulators
@@ -173,21 +174,31 @@ __device__ __forceinline__ uint32_t convert_pair16(uint32_t a0, uint32_t a1, flo
   return w;
 }
 
-// Stage one 32x32 box of 16-bit outputs ([32 rows m][32 columns n], 64 B
-// rows).  Lane n holds p[j] = (row 2j, row 2j+1) of column n.  Neighbour lanes
-// 2i and 2i+1 swap one half so that the even lane holds row 2j and the odd
-// lane row 2j+1 of the column pair (2i, 2i+1); every word lands in a distinct
-// bank (even lanes: banks i, odd lanes: banks 16+i).
-__device__ __forceinline__ void stage_box16(uint8_t* buf, const uint32_t (&p)[16], int lane) {
+// Stage this warp's half of a [32 rows m][64 columns n] box of 16-bit outputs
+// (128 B rows, 128-byte swizzle: 16-byte chunk c of row r sits at chunk
+// c ^ (r % 8); the box starts 1024-byte aligned); `half` selects columns
+// 32*half .. 32*half+31.  Lane n holds p[j] = (row 2j, row 2j+1) of column n.
+// At step j the even lane 2i stores row 2j and the odd lane 2i+1 row
+// 2(j^2)+1 of the column pair (2i, 2i+1), each taking the missing half from
+// its neighbour; with the swizzle the two halves of the warp always land in
+// disjoint bank groups.
+__device__ __forceinline__ void stage_pair_box16(uint32_t box_saddr, const uint32_t (&p)[16], int lane, int half) {
   const bool even = (lane & 1) == 0;
-  uint32_t* o = reinterpret_cast<uint32_t*>(buf) + (lane >> 1) + (even ? 0 : 16);
+  const int i = lane >> 1;
+  // unswizzled byte offset of this lane's word within its row
+  const uint32_t base = box_saddr + uint32_t(((4 * half + (i >> 2)) << 4) + (i & 3) * 4);
 #pragma unroll
   for (int j = 0; j < 16; ++j) {
-    // even lanes give away row 2j+1 (high half), odd lanes row 2j (low half)
-    const uint32_t send = even ? (p[j] >> 16) : (p[j] & 0xFFFFu);
+    const int jo = j ^ 2;
+    // the even lane stores row 2j and needs the odd lane's row 2j; the odd
+    // lane stores row 2jo+1 and needs the even lane's row 2jo+1
+    const uint32_t send = even ? (p[jo] >> 16) : (p[j] & 0xFFFFu);
     const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 1);
-    const uint32_t w = even ? __byte_perm(p[j], recv, 0x5410) : __byte_perm(recv, p[j], 0x7610);
-    o[j * 32] = w;  // row 2j (even) or 2j+1 (odd): 32 words = 2 rows of 64 B apart per j
+    const uint32_t w = even ? __byte_perm(p[j], recv, 0x5410) : __byte_perm(recv, p[jo], 0x7610);
+    const uint32_t re = 2 * j, ro = 2 * jo + 1;
+    const uint32_t ae = (base + re * 128) ^ ((re & 7) << 4);
+    const uint32_t ao = (base + ro * 128) ^ ((ro & 7) << 4);
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(even ? ae : ao), "r"(w) : "memory");
   }
 }
 
@@ -386,15 +397,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ---------------- epilogue (both CTAs) ----------------
-    // Warp w reads tensor-memory lanes 32*(w%4).. (its quadrant) and one half
-    // of the accumulator's 32-column chunks; the next chunk's tcgen05.ld is in
-    // flight while the current one is converted and stored.
+    // Warp w reads tensor-memory lanes 32*(w%4).. (its quadrant) and every
+    // second 32-column chunk of the accumulator, starting at chunk (w-4)/4.
+    constexpr int kStride = C::EPI_WARPS / 4;
     const int q = warp & 3;
-    const int half = (warp - 4) >> 2;
-    const int c_lo = half ? C::CH_HALF : 0;
-    const int c_hi = half ? C::NCH : C::CH_HALF;
-    uint8_t* epi = smem + C::OFF_EPI + (warp - 4) * 2 * C::EPI_BUF;
-    uint32_t cc = 0;  // output boxes staged by this warp so far
+    const int sub = (warp - 4) >> 2;
+    uint8_t* buf = smem + C::OFF_EPI + (warp - 4) * C::EPI_BUF;
+    // 16-bit outputs: warps (sub, 2p) and (sub, 2p+1) share two 4 KB pair boxes
+    const int pair_idx = (warp - 4) >> 1;
+    const uint32_t pbox0 = smem_addr(smem + C::OFF_EPI + pair_idx * 2 * C::EPI_BUF);
+    const uint32_t pair_bar = 1 + pair_idx;
+    const bool pair_lead = (q & 1) == 0;
+    bool staged = false;  // int32: a TMA store from buf may still be reading it
+    uint32_t nst = 0;     // 16-bit: pair boxes stored so far
     int i = 0;
     for (int t = pair; t < total; t += npairs, ++i) {
       const int n0 = (t % NT) * 256 + 128 * int(rank), m0 = (t / NT) * BN;
@@ -420,79 +435,79 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         }
       }
       const bool full_n = nb + 32 <= N;
+      const bool pair_full = n0 + 64 * (q >> 1) + 64 <= N;
       const uint32_t tbase = tmem + (uint32_t(32 * q) << 16) + uint32_t(b * BN);
-      if (c_lo >= c_hi) {  // narrow tiles: this warp has no chunk, only hands the accumulator back
+#pragma unroll 1
+      for (int c = sub; c < C::NCH; c += kStride) {
+        uint32_t h[32];
+        tmem_ld_32x32b_x32(tbase + 32 * c, h);
+        tmem_ld_wait(h);
+        if (c + kStride >= C::NCH) {
+          // last chunk of this warp is read: hand the accumulator back
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(acc_empty_l + 8u * b);
+        }
+        const int mb = m0 + 32 * c;
+        if (nb >= N || mb >= M) continue;
+        if constexpr (C::OUT_ES == 4) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) h[k] = convert_out<OUT, kInt8>(h[k], badd, sc, has_bias);
+        } else {
+          // packed pairs (rows 2j, 2j+1) kept in h[0..15]
+#pragma unroll
+          for (int j = 0; j < 16; ++j) h[j] = convert_pair16<OUT, kInt8>(h[2 * j], h[2 * j + 1], badd, sc, has_bias);
+        }
+        if (C::OUT_ES == 4 && full_n) {
+          // int32: one [32][32] box (128 B rows) per warp
+          if (staged) {
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int k = 0; k < 32; ++k) reinterpret_cast<uint32_t*>(buf)[k * 32 + lane] = h[k];
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmY, buf, nb, mb);
+            bulk_commit();
+          }
+          __syncwarp();
+          staged = true;
+        } else if (C::OUT_ES == 2 && pair_full) {
+          // 16-bit: the warps of quadrants 2p, 2p+1 fill one [32][64] box (128 B
+          // rows) of a double-buffered pair; the lead warp stores it
+          const uint32_t box = pbox0 + (nst & 1) * 4096;
+          if (nst >= 2) {
+            if (pair_lead && lane == 0) bulk_wait_read<1>();
+            named_bar_sync(pair_bar, 64);
+          }
+          stage_pair_box16(box, reinterpret_cast<const uint32_t(&)[16]>(h), lane, q & 1);
+          fence_proxy_async_smem();
+          named_bar_sync(pair_bar, 64);
+          if (pair_lead && lane == 0) {
+            tma_store_2d_saddr(&tmY, box, n0 + 64 * (q >> 1), mb);
+            bulk_commit();
+          }
+          __syncwarp();
+          ++nst;
+        } else if (n < N) {
+          // ragged right edge: bounds-checked direct stores
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            if (mb + k >= M) continue;
+            if constexpr (C::OUT_ES == 4)
+              static_cast<uint32_t*>(Yp)[int64_t(mb + k) * ldy + n] = h[k];
+            else
+              static_cast<uint16_t*>(Yp)[int64_t(mb + k) * ldy + n] =
+                  static_cast<uint16_t>((k & 1) ? (h[k >> 1] >> 16) : (h[k >> 1] & 0xFFFFu));
+          }
+        }
+      }
+      if (sub >= C::NCH) {  // narrow tiles: this warp has no chunk, only hands the accumulator back
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(acc_empty_l + 8u * b);
-        continue;
-      }
-      uint32_t r[2][32];
-      tmem_ld_32x32b_x32(tbase + 32 * c_lo, r[0]);
-      tmem_ld_wait(r[0]);
-#pragma unroll 1
-      for (int c = c_lo; c < c_hi; c += 2) {
-        // two chunks per iteration so that register indices stay static
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int cu = c + u;
-          if (cu >= c_hi) break;
-          const bool more = cu + 1 < c_hi;
-          if (more) tmem_ld_32x32b_x32(tbase + 32 * (cu + 1), r[u ^ 1]);
-          const int mb = m0 + 32 * cu;
-          if (nb < N && mb < M) {
-            uint32_t (&h)[32] = r[u];
-            if constexpr (C::OUT_ES == 4) {
-#pragma unroll
-              for (int k = 0; k < 32; ++k) h[k] = convert_out<OUT, kInt8>(h[k], badd, sc, has_bias);
-            } else {
-              // packed pairs (rows 2j, 2j+1) kept in h[0..15]
-#pragma unroll
-              for (int j = 0; j < 16; ++j) h[j] = convert_pair16<OUT, kInt8>(h[2 * j], h[2 * j + 1], badd, sc, has_bias);
-            }
-            if (full_n) {
-              if (cc >= 2) {
-                if (lane == 0) bulk_wait_read<1>();
-                __syncwarp();
-              }
-              uint8_t* buf = epi + (cc & 1) * C::EPI_BUF;
-              if constexpr (C::OUT_ES == 4) {
-#pragma unroll
-                for (int k = 0; k < 32; ++k) reinterpret_cast<uint32_t*>(buf)[k * 32 + lane] = h[k];
-              } else {
-                stage_box16(buf, reinterpret_cast<const uint32_t(&)[16]>(h), lane);
-              }
-              fence_proxy_async_smem();
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_2d(&tmY, buf, nb, mb);
-                bulk_commit();
-              }
-              __syncwarp();
-              ++cc;
-            } else if (n < N) {
-              // ragged right edge: bounds-checked direct stores
-#pragma unroll
-              for (int k = 0; k < 32; ++k) {
-                if (mb + k >= M) continue;
-                if constexpr (C::OUT_ES == 4)
-                  static_cast<uint32_t*>(Yp)[int64_t(mb + k) * ldy + n] = h[k];
-                else
-                  static_cast<uint16_t*>(Yp)[int64_t(mb + k) * ldy + n] =
-                      static_cast<uint16_t>((k & 1) ? (h[k >> 1] >> 16) : (h[k >> 1] & 0xFFFFu));
-              }
-            }
-          }
-          if (more) {
-            tmem_ld_wait(r[u ^ 1]);
-          }
-          if (cu + 1 == c_hi) {
-            // every chunk of this warp is read: hand the accumulator back
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc_empty_l + 8u * b);
-          }
-        }
       }
     }
     if (lane == 0) bulk_wait_all<0>();
@@ -551,7 +566,8 @@ spg_status launch(const void* X, int64_t ldx, const void* Wv, const uint8_t* met
   if (!make_tmap_2d(&tmA, Wv, es, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2) * es, 128 / es, 128, true) ||
       !make_tmap_2d(&tmB, X, es, uint64_t(K), uint64_t(M), uint64_t(ldx) * es, 128 / es, C::BNH, true) ||
       !make_tmap_2d(&tmE, meta, 1, uint64_t(K / 8), uint64_t(N), uint64_t(K / 8), 16, 128, false) ||
-      !make_tmap_2d(&tmY, Y, C::OUT_ES, uint64_t(N), uint64_t(M), uint64_t(ldy) * C::OUT_ES, 32, 32, false))
+      !make_tmap_2d(&tmY, Y, C::OUT_ES, uint64_t(N), uint64_t(M), uint64_t(ldy) * C::OUT_ES,
+                    C::OUT_ES == 2 ? 64 : 32, 32, C::OUT_ES == 2))
     return SPG_ERR_CUDA;
   uint32_t* err = device_error_word();
   if (!err) return SPG_ERR_CUDA;
