@@ -175,8 +175,9 @@ spg_status spgemm_24_s8(const int8_t* X, int64_t ldx, const int8_t* Wv, const ui
 typedef struct {
   int64_t N, K, Nk;
   int32_t G, T;
-  int64_t offsetk_len; /* tile_kofs[T] */
-  int64_t wc_elems;    /* offsetk_len * G */
+  int64_t offsetk_len;    /* tile_kofs[T] */
+  int64_t wc_elems;       /* offsetk_len * G */
+  int64_t reorg_ws_bytes; /* device workspace tw_reorganize needs (exact column norms) */
 } spg_tw_sizes;
 
 typedef struct {
@@ -191,18 +192,22 @@ typedef struct {
   void* Wc; /* fp16 */
 } spg_tw_desc;
 
-/* Sizes of the descriptor buffers.  k_per_tile is a HOST array of T entries
- * (T = ceil((N - n_pruned) / G)), each in [1, K].  G must be 128; 0 <=
- * n_pruned < N; K % 64 == 0. */
+/* Sizes of the descriptor buffers and of the reorganisation workspace.
+ * k_per_tile is a HOST array of T entries (T = ceil((N - n_pruned) / G)),
+ * each in [1, K].  G must be 128; 0 <= n_pruned < N; K % 64 == 0 and
+ * K <= 8192; N < 2^31. */
 spg_status tw_query_sizes(int64_t N, int64_t K, int32_t G, int64_t n_pruned, const int32_t* k_per_tile,
                           spg_tw_sizes* out);
 
 /* Fill `desc` (whose sizes and device pointers the caller set; sizes must
- * equal tw_query_sizes) from the dense fp16 W [N, K] (pitch ldw, 16-byte
- * aligned rows).  k_per_tile is a HOST array of T entries.  The integer
- * outputs are exact (bit-identical to the selection rule above). */
+ * equal tw_query_sizes) from the dense fp16 W [N, K] (pitch ldw >= K,
+ * 2-byte aligned).  k_per_tile is a HOST array of T entries; it is copied
+ * to the device before the call returns.  `workspace` (device, 16-byte
+ * aligned, ws_bytes >= reorg_ws_bytes) holds the exact column norms; its
+ * contents are scratch.  The integer outputs are exact (bit-identical to the
+ * selection rule above). */
 spg_status tw_reorganize(const void* W, int64_t ldw, int64_t n_pruned, const int32_t* k_per_tile,
-                         const spg_tw_desc* desc, spg_stream_t stream);
+                         const spg_tw_desc* desc, void* workspace, size_t ws_bytes, spg_stream_t stream);
 
 /* Workspace bytes spgemm_tw_f16 needs: M*K*2 (rounded up to 256) for
  * x_layout SPG_X_MK (the transposed activations), 0 for SPG_X_KM. */
@@ -215,9 +220,9 @@ size_t tw_workspace_size(int64_t M, int64_t K, int x_layout);
  * [K, M] pitch ldx (SPG_X_KM: the transpose is assumed fused upstream).  Y
  * fp16 [M, N] pitch ldy; every element of Y is written (pruned columns +0).
  * fp32 accumulation, one round-to-nearest-even.
- * Limits: M % 8 == 0 (the [K, M] rows are TMA rows), M >= 8; X, Y, workspace
- * 16-byte aligned, ldx and ldy multiples of 8; ws_bytes >=
- * tw_workspace_size(M, K, x_layout). */
+ * Limits: M % 8 == 0 (the [K, M] rows are TMA rows), M >= 8; X and
+ * workspace 16-byte aligned, ldx a multiple of 8; Y 2-byte aligned, any
+ * ldy >= N; ws_bytes >= tw_workspace_size(M, K, x_layout). */
 spg_status spgemm_tw_f16(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Y,
                          int64_t ldy, int64_t M, void* workspace, size_t ws_bytes, spg_stream_t stream);
 

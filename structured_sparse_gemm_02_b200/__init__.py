@@ -31,7 +31,7 @@ _i64, _i32, _p, _sz = ctypes.c_int64, ctypes.c_int32, ctypes.c_void_p, ctypes.c_
 
 class SpgTwSizes(ctypes.Structure):
     _fields_ = [("N", _i64), ("K", _i64), ("Nk", _i64), ("G", _i32), ("T", _i32),
-                ("offsetk_len", _i64), ("wc_elems", _i64)]
+                ("offsetk_len", _i64), ("wc_elems", _i64), ("reorg_ws_bytes", _i64)]
 
 
 class SpgTwDesc(ctypes.Structure):
@@ -49,7 +49,8 @@ SIGNATURES = {
     "spgemm_24_f16": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_s8": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _p, _i64, ctypes.c_int, _i64, _i64, _i64, _p]),
     "tw_query_sizes": (ctypes.c_int, [_i64, _i64, _i32, _i64, ctypes.POINTER(_i32), ctypes.POINTER(SpgTwSizes)]),
-    "tw_reorganize": (ctypes.c_int, [_p, _i64, _i64, ctypes.POINTER(_i32), ctypes.POINTER(SpgTwDesc), _p]),
+    "tw_reorganize": (ctypes.c_int, [_p, _i64, _i64, ctypes.POINTER(_i32), ctypes.POINTER(SpgTwDesc), _p, _sz,
+                                     _p]),
     "tw_workspace_size": (_sz, [_i64, _i64, ctypes.c_int]),
     "spgemm_tw_f16": (ctypes.c_int, [_p, _i64, ctypes.c_int, ctypes.POINTER(SpgTwDesc), _p, _i64, _i64, _p,
                                      _sz, _p]),
@@ -187,12 +188,15 @@ class TwDesc:
                            self.offsetk.data_ptr(), self.Wc.data_ptr())
 
 
-def tw_reorganize(W, G: int, n_pruned: int, k_per_tile: Sequence[int], stream=None) -> TwDesc:
+def tw_reorganize(W, G: int, n_pruned: int, k_per_tile: Sequence[int], workspace=None, stream=None) -> TwDesc:
     """Condense a dense fp16 W [N, K] into a tile-wise descriptor."""
+    import torch
     N, K = W.shape
     d = TwDesc(N, K, G, n_pruned, k_per_tile, device=W.device)
+    if workspace is None:
+        workspace = torch.empty(max(16, d.sizes.reorg_ws_bytes), dtype=torch.uint8, device=W.device)
     _check("tw_reorganize", lib().tw_reorganize(_ptr(W), W.stride(0), n_pruned, d.k_host, ctypes.byref(d.c),
-                                                _stream(stream)))
+                                                _ptr(workspace), workspace.numel(), _stream(stream)))
     return d
 
 

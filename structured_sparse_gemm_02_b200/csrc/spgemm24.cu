@@ -320,7 +320,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       for (int t = pair; ok && t < total; t += npairs) {
         for (int kb = 0; kb < KB; ++kb, ++g) {
           const int s = g % STAGES;
-          if (!mbar_wait(&mtma[s], (g / STAGES) & 1, abort_flag, err, ERR_WAIT_META)) {
+          if (!mbar_wait_warp(&mtma[s], (g / STAGES) & 1, abort_flag, err, ERR_WAIT_META)) {
             ok = false;
             break;
           }
@@ -341,18 +341,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       bool ok = true;
       for (int t = pair; ok && t < total; t += npairs, ++i) {
         const int b = i & 1;
-        if (i >= 2 && !mbar_wait(&acc_empty[b], ((i >> 1) - 1) & 1, abort_flag, err, ERR_WAIT_ACC_FREE)) break;
+        if (i >= 2 && !mbar_wait_warp(&acc_empty[b], ((i >> 1) - 1) & 1, abort_flag, err, ERR_WAIT_ACC_FREE)) break;
         tc_fence_after();
         const uint32_t acc = tmem + uint32_t(b * BN);
         for (int kb = 0; kb < KB; ++kb, ++g) {
           const int s = g % STAGES;
           const uint32_t ph = (g / STAGES) & 1;
-          if (!mbar_wait(&full[s], ph, abort_flag, err, ERR_WAIT_FULL)) {
+          if (!mbar_wait_warp(&full[s], ph, abort_flag, err, ERR_WAIT_FULL)) {
             ok = false;
             break;
           }
           if constexpr (!kInt8) {
-            if (!mbar_wait(&meta_full[s], ph, abort_flag, err, ERR_WAIT_META)) {
+            if (!mbar_wait_warp(&meta_full[s], ph, abort_flag, err, ERR_WAIT_META)) {
               ok = false;
               break;
             }
@@ -414,7 +414,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     for (int t = pair; t < total; t += npairs, ++i) {
       const int n0 = (t % NT) * 256 + 128 * int(rank), m0 = (t / NT) * BN;
       const int b = i & 1;
-      if (!mbar_wait(&acc_full[b], (i >> 1) & 1, abort_flag, err, ERR_WAIT_ACC)) break;
+      if (!mbar_wait_warp(&acc_full[b], (i >> 1) & 1, abort_flag, err, ERR_WAIT_ACC)) break;
       tc_fence_after();
       const int nb = n0 + 32 * q;
       const int n = nb + lane;

@@ -1,26 +1,510 @@
 // Tile-wise sparsity ("Accelerating Sparse DNN Models without Hardware-Support
-// via Tile-Wise Sparsity", slides "Tile-Wise Sparsity", "Re-organize",
-// "Run-time", "Transpose"): descriptor sizing.
+// via Tile-Wise Sparsity", Guo et al.): the offline reorganisation of a dense
+// fp16 W into condensed tiles (slides "Tile-Wise Sparsity", "Re-organize",
+// "Preprocessed"), the explicit activation transpose (slide "Transpose") and
+// the run-time GEMM that gathers A through offsetk and scatters C through
+// offsetn (slide "Run-time").
+//
+// In C = A x B of the slides, A = X [M, K], B = W^T and C = Y [M, N]: the
+// columns of B are the rows n of W, its rows the reduction indices k.
+#include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <vector>
 
 #include "host.cuh"
+#include "sm100.cuh"
 #include "spgemm.h"
 
 namespace spg {
 namespace tw {
 
+using u128 = unsigned __int128;
+
+constexpr int kG = 128;          // tile width (kept columns per tile)
+constexpr int kKBlock = 64;      // K padding / GEMM K block
+constexpr int kMaxK = 8192;      // reorganisation keeps a tile's K row norms in shared memory
+
+// ---- exact norms ------------------------------------------------------------------------
+// An fp16 value is +-m * 2^e with m = 1024 + frac, e = exp - 25 (normal) or
+// m = frac, e = -24 (subnormal), so w*w*2^48 = m*m * 2^(2e+48) is an integer
+// with 2e+48 = 2*exp - 2 (normal) or 0 (subnormal).  Sums of these are exact
+// in 128 bits (each term < 2^82, at most 2^31 terms) and order independent.
+__device__ __forceinline__ u128 sq_units(uint32_t bits) {
+  const uint32_t ex = (bits >> 10) & 0x1Fu, fr = bits & 0x3FFu;
+  const uint32_t m = ex ? (fr | 0x400u) : fr;
+  const uint32_t sh = ex ? 2u * ex - 2u : 0u;
+  return static_cast<u128>(static_cast<uint64_t>(m) * m) << sh;
+}
+
+__device__ __forceinline__ u128 shfl_xor_u128(u128 v, int mask) {
+  const uint64_t lo = static_cast<uint64_t>(v), hi = static_cast<uint64_t>(v >> 64);
+  const uint64_t l2 = __shfl_xor_sync(0xffffffffu, lo, mask), h2 = __shfl_xor_sync(0xffffffffu, hi, mask);
+  return (static_cast<u128>(h2) << 64) | l2;
+}
+
+// Column keys: key[n] = sum_k w[n][k]^2 (x 2^48), one warp per row n of W.
+__global__ void col_keys_kernel(const uint16_t* __restrict__ W, int64_t ldw, int N, int K, u128* __restrict__ keys) {
+  const int lane = threadIdx.x & 31;
+  const int wpb = blockDim.x >> 5;
+  for (int n = blockIdx.x * wpb + (threadIdx.x >> 5); n < N; n += gridDim.x * wpb) {
+    const uint16_t* row = W + int64_t(n) * ldw;
+    u128 acc = 0;
+    for (int k = lane; k < K; k += 32) acc += sq_units(row[k]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += shfl_xor_u128(acc, o);
+    if (lane == 0) keys[n] = acc;
+  }
+}
+
+// Column n is pruned when fewer than P columns precede it in the order
+// (key ascending, index ascending), i.e. it is among the P smallest.
+__global__ void col_prune_kernel(const u128* __restrict__ keys, int N, int P, int* __restrict__ kept) {
+  __shared__ u128 sk[1024];
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  const u128 mine = n < N ? keys[n] : 0;
+  int before = 0;
+  for (int base = 0; base < N; base += 1024) {
+    const int cnt = min(1024, N - base);
+    __syncthreads();
+    for (int i = threadIdx.x; i < cnt; i += blockDim.x) sk[i] = keys[base + i];
+    __syncthreads();
+    if (n < N)
+      for (int i = 0; i < cnt; ++i) {
+        const u128 o = sk[i];
+        before += (o < mine) || (o == mine && base + i < n);
+      }
+  }
+  if (n < N) kept[n] = before >= P ? 1 : 0;
+}
+
+// Block-wide exclusive scan of 0/1 flags in chunks of blockDim.x; calls
+// emit(i, position) for every set flag i in ascending order.  One CTA.
+template <typename Flag, typename Emit>
+__device__ void compact_ascending(Flag flag, int count, int* s_warp, Emit emit) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  int carry = 0;
+  for (int base = 0; base < count; base += blockDim.x) {
+    const int i = base + tid;
+    const int f = (i < count && flag(i)) ? 1 : 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, f);
+    const int in_warp = __popc(bal & ((1u << lane) - 1u));
+    if (lane == 0) s_warp[warp] = __popc(bal);
+    __syncthreads();
+    int warp_off = 0, total = 0;
+    for (int w = 0; w < nw; ++w) {
+      if (w < warp) warp_off += s_warp[w];
+      total += s_warp[w];
+    }
+    if (f) emit(i, carry + warp_off + in_warp);
+    carry += total;
+    __syncthreads();
+  }
+}
+
+// offsetn (kept columns ascending) and tile_n0 (output column range of each tile).
+__global__ void col_compact_kernel(const int* __restrict__ kept, int N, int T, int* __restrict__ offsetn,
+                                   int* __restrict__ tile_n0) {
+  __shared__ int s_warp[32];
+  compact_ascending([&](int i) { return kept[i] != 0; }, N, s_warp,
+                    [&](int i, int pos) {
+                      offsetn[pos] = i;
+                      if (pos % kG == 0) tile_n0[pos / kG] = pos == 0 ? 0 : i;
+                    });
+  if (threadIdx.x == 0) tile_n0[T] = N;
+}
+
+// One CTA per tile: exact row keys over the tile's kept columns, the k_t
+// largest (ties: lower k first) kept, offsetk written ascending and padded to
+// a multiple of 64 with the last kept k.
+__global__ void tile_rows_kernel(const uint16_t* __restrict__ W, int64_t ldw, int K, int Nk,
+                                 const int* __restrict__ offsetn, const int* __restrict__ tile_kofs,
+                                 const int* __restrict__ k_per_tile, int* __restrict__ offsetk) {
+  extern __shared__ uint8_t sm_raw[];
+  u128* keys = reinterpret_cast<u128*>(sm_raw);
+  int* keep = reinterpret_cast<int*>(keys + K);
+  __shared__ int s_warp[32];
+  __shared__ int s_last;
+  const int t = blockIdx.x;
+  const int j0 = t * kG;
+  const int Gt = min(kG, Nk - j0);
+  const int kt = k_per_tile[t];
+  const int kofs = tile_kofs[t];
+  const int kpad = tile_kofs[t + 1] - kofs;
+  for (int k = threadIdx.x; k < K; k += blockDim.x) keys[k] = 0;
+  __syncthreads();
+  for (int j = 0; j < Gt; ++j) {
+    const uint16_t* row = W + int64_t(offsetn[j0 + j]) * ldw;
+    for (int k = threadIdx.x; k < K; k += blockDim.x) keys[k] += sq_units(row[k]);
+  }
+  __syncthreads();
+  for (int k = threadIdx.x; k < K; k += blockDim.x) {
+    const u128 mine = keys[k];
+    int before = 0;
+    for (int o = 0; o < K; ++o) {
+      const u128 v = keys[o];
+      before += (v > mine) || (v == mine && o < k);
+    }
+    keep[k] = before < kt ? 1 : 0;
+  }
+  __syncthreads();
+  compact_ascending([&](int i) { return keep[i] != 0; }, K, s_warp, [&](int i, int pos) {
+    offsetk[kofs + pos] = i;
+    if (pos == kt - 1) s_last = i;
+  });
+  __syncthreads();
+  for (int i = kt + threadIdx.x; i < kpad; i += blockDim.x) offsetk[kofs + i] = s_last;
+}
+
+// Condensed values, block b of tile t: Wc[blk][j][c] = W[offsetn[tG+j]][offsetk[kofs+64b+c]].
+__global__ void gather_wc_kernel(const uint16_t* __restrict__ W, int64_t ldw, int Nk,
+                                 const int* __restrict__ offsetn, const int* __restrict__ tile_kofs,
+                                 const int* __restrict__ k_per_tile, const int* __restrict__ offsetk,
+                                 uint16_t* __restrict__ Wc) {
+  const int t = blockIdx.x, b = blockIdx.y;
+  const int kofs = tile_kofs[t];
+  if (b * kKBlock >= tile_kofs[t + 1] - kofs) return;
+  const int j0 = t * kG;
+  const int Gt = min(kG, Nk - j0);
+  const int kt = k_per_tile[t];
+  uint16_t* out = Wc + (int64_t(kofs / kKBlock + b) * kG) * kKBlock;
+  for (int e = threadIdx.x; e < kG * kKBlock; e += blockDim.x) {
+    const int j = e / kKBlock, c = e % kKBlock;
+    const int i = b * kKBlock + c;
+    uint16_t v = 0;
+    if (j < Gt && i < kt) v = W[int64_t(offsetn[j0 + j]) * ldw + offsetk[kofs + i]];
+    out[e] = v;
+  }
+}
+
+// ---- explicit activation transpose X [M, K] -> Xt [K, M] ------------------------------------
+// 64 x 64 tiles through shared memory; 32-bit (two fp16) accesses on both sides.
+__global__ void transpose_kernel(const uint16_t* __restrict__ X, int64_t ldx, int M, int K,
+                                 uint16_t* __restrict__ Xt, int64_t ldt) {
+  __shared__ uint32_t tile[64][33];  // [m][k pair]
+  const int m0 = blockIdx.y * 64, k0 = blockIdx.x * 64;
+  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int m = m0 + ty + 8 * r, k = k0 + 2 * tx;
+    uint32_t v = 0;
+    if (m < M && k + 1 < K) {
+      v = *reinterpret_cast<const uint32_t*>(X + int64_t(m) * ldx + k);
+    } else if (m < M && k < K) {
+      v = X[int64_t(m) * ldx + k];
+    }
+    tile[ty + 8 * r][tx] = v;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < 8; ++r) {
+    const int kl = ty + 8 * r, k = k0 + kl;
+    const int m = m0 + 2 * tx;
+    if (k >= K || m >= M) continue;
+    const int sh = 16 * (kl & 1);
+    const uint32_t lo = (tile[2 * tx][kl >> 1] >> sh) & 0xFFFFu;
+    const uint32_t hi = (tile[2 * tx + 1][kl >> 1] >> sh) & 0xFFFFu;
+    if (m + 1 < M)
+      *reinterpret_cast<uint32_t*>(Xt + int64_t(k) * ldt + m) = lo | (hi << 16);
+    else
+      Xt[int64_t(k) * ldt + m] = static_cast<uint16_t>(lo);
+  }
+}
+
+// ---- run-time GEMM -------------------------------------------------------------------------
+// Work unit (tile t, 128-row block of X): D[j][m] = sum_i Wc_t[j][i] * X[m][offsetk_t[i]]
+// on the dense tensor cores (A = condensed tile, K-major; B = gathered rows of
+// Xt, MN-major), then Y[m][offsetn[tG+j]] = D[j][m] and +0 in the tile's
+// pruned columns.  Persistent CTAs, warp 0 loads (TMA for the tile block,
+// 16-byte cp.async per lane for the kept rows of Xt), warp 2 issues
+// tcgen05.mma into one of two accumulators, warps 4-7 drain, stage the
+// tile's output span in shared memory and write whole rows of Y.
+constexpr int BN = 128;                   // X rows per work unit
+constexpr int A_BYTES = kG * kKBlock * 2;  // 16 KB
+constexpr int B_BYTES = kKBlock * BN * 2;  // 16 KB: 64 gathered rows x 128 m, two 64-wide atoms
+constexpr int STAGES = 4;
+constexpr int MAX_SPAN = 256;              // widest tile output span staged in shared memory
+constexpr int OFF_STG = STAGES * (A_BYTES + B_BYTES);
+constexpr int OFF_BAR = OFF_STG + BN * MAX_SPAN * 2;
+constexpr int SMEM = OFF_BAR + (2 * STAGES + 5) * 8 + 16 + 1024;
+static_assert(SMEM <= 232448, "shared memory budget");
+constexpr uint32_t TMEM_COLS = 256;
+
+__device__ __forceinline__ void tail_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  int never = 0;
+  mbar_wait(bar, parity, &never, err, ERR_WAIT_TAIL);
+}
+
+// 16-byte global -> shared copy; src_bytes 0 fills the destination with zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+// Arrive on `bar` once every cp.async issued so far by this thread has landed.
+__device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_addr(bar)) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+__global__ void __launch_bounds__(256, 1)
+    tw_gemm_kernel(const __grid_constant__ CUtensorMap tmWc, const uint16_t* __restrict__ xt, int64_t ldt,
+                   uint16_t* __restrict__ Y, int64_t ldy, int M, int Nk, int T, const int* __restrict__ offsetn,
+                   const int* __restrict__ tile_n0, const int* __restrict__ tile_kofs,
+                   const int* __restrict__ offsetk, uint32_t* err) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
+  uint64_t* empty = full + STAGES;
+  uint64_t* acc_full = empty + STAGES;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* mma_done = acc_empty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int MB = (M + BN - 1) / BN;
+  const int units = T * MB;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 33);  // TMA of the tile block + one cp.async arrival per producer lane
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmWc);
+  if (warp == 2) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if (warp == 0) {
+    // ---------------- loads ----------------
+    // The 64 row indices of a K block are read by the whole warp (two per
+    // lane) one block ahead of their use; lane 0 issues the copies.
+    uint32_t g = 0;
+    bool ok = true;
+    int u = blockIdx.x;
+    int kb = 0;
+    // indices of the next block to issue
+    int nxt0 = 0, nxt1 = 0;
+    auto load_idx = [&](int uu, int kk) {
+      if (uu < units) {
+        const int* rows = offsetk + tile_kofs[uu / MB] + kk * kKBlock;
+        nxt0 = rows[lane];
+        nxt1 = rows[32 + lane];
+      }
+    };
+    load_idx(u, 0);
+    while (ok && u < units) {
+      const int t = u / MB, mb = (u % MB) * BN;
+      const int kofs = tile_kofs[t];
+      const int KB = (tile_kofs[t + 1] - kofs) / kKBlock;
+      const int cur0 = nxt0, cur1 = nxt1;
+      // advance to the following block and prefetch its indices
+      int un = u, kn = kb + 1;
+      if (kn == KB) {
+        un = u + gridDim.x;
+        kn = 0;
+      }
+      load_idx(un, kn);
+      const int s = g % STAGES;
+      const uint32_t use = g / STAGES;
+      if (use > 0 && !mbar_wait_warp(&empty[s], (use - 1) & 1, abort_flag, err, ERR_WAIT_EMPTY)) {
+        ok = false;
+        break;
+      }
+      uint8_t* a_s = smem + s * (A_BYTES + B_BYTES);
+      const uint32_t b_s = smem_addr(a_s + A_BYTES);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&full[s], A_BYTES);
+        tma_load_2d(a_s, &tmWc, 0, (kofs / kKBlock + kb) * kG, &full[s]);
+      }
+      // B: the 64 kept rows of Xt for this block, 128 m each, as two MN-major
+      // 128-byte-swizzled atoms of 64 m (chunk c of row r at chunk c ^ (r % 8))
+      const int a = (lane >> 3) & 1, c = lane & 7;
+      const int mcol = mb + 64 * a + 8 * c;
+      const uint32_t src_bytes = mcol < M ? 16u : 0u;
+#pragma unroll
+      for (int i = 0; i < kKBlock / 2; ++i) {
+        const int r = 2 * i + (lane >> 4);
+        const int rk = __shfl_sync(0xffffffffu, i < 16 ? cur0 : cur1, r & 31);
+        const uint32_t dst = b_s + a * 8192 + r * 128 + ((c ^ (r & 7)) << 4);
+        cp_async16(dst, xt + int64_t(rk) * ldt + (src_bytes ? mcol : 0), src_bytes);
+      }
+      cp_async_arrive(&full[s]);
+      ++g;
+      u = un;
+      kb = kn;
+    }
+    cp_async_wait_all();
+    if (lane == 0)
+      for (uint32_t q = (g > uint32_t(STAGES) ? g - STAGES : 0u); q < g; ++q)
+        tail_wait(&full[q % STAGES], (q / STAGES) & 1, err);
+    __syncwarp();
+  } else if (warp == 2) {
+    // ---------------- MMA ----------------
+    // kind::f16 dense, fp16 inputs, fp32 accumulate, A K-major, B MN-major, M=128, N=128
+    constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | ((BN >> 3) << 17) | ((128 >> 4) << 24);
+    uint32_t g = 0;
+    int i = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++i) {
+      const int t = u / MB;
+      const int KB = (tile_kofs[t + 1] - tile_kofs[t]) / kKBlock;
+      const int b = i & 1;
+      if (i >= 2 && !mbar_wait_warp(&acc_empty[b], ((i >> 1) - 1) & 1, abort_flag, err, ERR_WAIT_ACC_FREE)) break;
+      tc_fence_after();
+      const uint32_t acc = tmem + uint32_t(b * BN);
+      for (int kb = 0; kb < KB; ++kb, ++g) {
+        const int s = g % STAGES;
+        if (!mbar_wait_warp(&full[s], (g / STAGES) & 1, abort_flag, err, ERR_WAIT_FULL)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        fence_proxy_async_smem();  // the gathered rows were written by cp.async (generic proxy)
+        if (lane == 0) {
+          const uint32_t a_s = smem_addr(smem + s * (A_BYTES + B_BYTES));
+          const uint32_t b_s = a_s + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < kKBlock / 16; ++kk) {
+            const uint64_t adesc = smem_desc(a_s + 32 * kk, 16, 1024, LAYOUT_SW128);
+            const uint64_t bdesc = smem_desc(b_s + 2048 * kk, 8192, 1024, LAYOUT_SW128);
+            tc_mma(acc, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+          }
+          tc_commit(&empty[s]);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) tc_commit(&acc_full[b]);
+      __syncwarp();
+    }
+    if (lane == 0) {
+      tc_commit(mma_done);
+      tail_wait(mma_done, 0, err);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // ---------------- drain and scatter ----------------
+    const int q = warp & 3;
+    int i = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
+      const int t = u / MB, mb = (u % MB) * BN;
+      const int b = i & 1;
+      if (!mbar_wait_warp(&acc_full[b], (i >> 1) & 1, abort_flag, err, ERR_WAIT_ACC)) break;
+      tc_fence_after();
+      uint32_t r[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld_32x32b_x32(tmem + (uint32_t(32 * q) << 16) + uint32_t(b * BN + 32 * c), r[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
+
+      const int j0 = t * kG;
+      const int Gt = min(kG, Nk - j0);
+      const int j = 32 * q + lane;
+      const bool valid = j < Gt;
+      const int nj = valid ? offsetn[j0 + j] : 0;
+      const int n0 = tile_n0[t], n1 = tile_n0[t + 1];
+      const int span = n1 - n0;
+      // pruned columns owned by this lane: the gap after its kept column, and
+      // for the first kept column of the tile also the gap before it
+      const int gap_end = valid ? (j + 1 < Gt ? offsetn[j0 + j + 1] : n1) : 0;
+      const int lead0 = (valid && j == 0) ? n0 : 0;
+      const int lead1 = (valid && j == 0) ? nj : 0;
+      const int rows = min(BN, M - mb);
+      if (span <= MAX_SPAN) {
+        // stage the output rows of the span (kept values and zeros) and write
+        // every row of Y contiguously
+        uint16_t* stg = reinterpret_cast<uint16_t*>(smem + OFF_STG);
+        named_bar_sync(1, 128);  // the previous unit's rows have been written out
+        if (valid) {
+          const int col = nj - n0;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              stg[(32 * cc + k) * MAX_SPAN + col] = __half_as_ushort(__float2half_rn(__uint_as_float(r[cc][k])));
+          if (gap_end > nj + 1 || lead1 > lead0) {
+#pragma unroll 1
+            for (int k = 0; k < BN; ++k) {
+              for (int z = nj + 1; z < gap_end; ++z) stg[k * MAX_SPAN + z - n0] = 0;
+              for (int z = lead0; z < lead1; ++z) stg[k * MAX_SPAN + z - n0] = 0;
+            }
+          }
+        }
+        named_bar_sync(1, 128);
+#pragma unroll 1
+        for (int k = q * 32; k < q * 32 + 32; ++k) {
+          if (k >= rows) break;
+          uint16_t* yrow = Y + int64_t(mb + k) * ldy + n0;
+          const uint16_t* srow = stg + k * MAX_SPAN;
+          for (int cidx = lane; cidx < span; cidx += 32) yrow[cidx] = srow[cidx];
+        }
+      } else {
+        // very wide span: direct stores
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const int m = mb + 32 * cc + k;
+            if (valid && m < M)
+              Y[int64_t(m) * ldy + nj] = __half_as_ushort(__float2half_rn(__uint_as_float(r[cc][k])));
+          }
+        }
+        if (valid && (gap_end > nj + 1 || lead1 > lead0)) {
+#pragma unroll 1
+          for (int k = 0; k < rows; ++k) {
+            uint16_t* yrow = Y + int64_t(mb + k) * ldy;
+            for (int z = nj + 1; z < gap_end; ++z) yrow[z] = 0;
+            for (int z = lead0; z < lead1; ++z) yrow[z] = 0;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+int sm_count() {
+  int dev = 0, v = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+  return v;
+}
+
 spg_status query(int64_t N, int64_t K, int32_t G, int64_t n_pruned, const int32_t* kpt, spg_tw_sizes* out) {
   if (!kpt || !out) return SPG_ERR_INVALID_ARG;
   if (N <= 0 || K <= 0 || n_pruned < 0 || n_pruned >= N) return SPG_ERR_INVALID_ARG;
-  if (G != 128 || K % 64 || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
+  if (G != kG || K % kKBlock || K > kMaxK || N >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
   const int64_t Nk = N - n_pruned;
   const int64_t T = (Nk + G - 1) / G;
   int64_t kofs = 0;
   for (int64_t t = 0; t < T; ++t) {
     if (kpt[t] < 1 || kpt[t] > K) return SPG_ERR_INVALID_ARG;
-    kofs += (kpt[t] + 63) / 64 * 64;
+    kofs += (kpt[t] + kKBlock - 1) / kKBlock * kKBlock;
   }
   out->N = N;
   out->K = K;
@@ -29,6 +513,7 @@ spg_status query(int64_t N, int64_t K, int32_t G, int64_t n_pruned, const int32_
   out->T = static_cast<int32_t>(T);
   out->offsetk_len = kofs;
   out->wc_elems = kofs * G;
+  out->reorg_ws_bytes = (N * 16 + N * 4 + 255) / 256 * 256;
   return SPG_OK;
 }
 
@@ -48,16 +533,91 @@ size_t tw_workspace_size(int64_t M, int64_t K, int x_layout) {
 }
 
 spg_status tw_reorganize(const void* W, int64_t ldw, int64_t n_pruned, const int32_t* k_per_tile,
-                         const spg_tw_desc* desc, spg_stream_t stream) {
-  (void)W; (void)ldw; (void)n_pruned; (void)k_per_tile; (void)desc; (void)stream;
-  return SPG_ERR_UNSUPPORTED_SHAPE;
+                         const spg_tw_desc* desc, void* workspace, size_t ws_bytes, spg_stream_t stream) {
+  using namespace spg;
+  using namespace spg::tw;
+  if (!W || !desc || !k_per_tile || !workspace) return SPG_ERR_INVALID_ARG;
+  spg_tw_sizes sz{};
+  spg_status st = query(desc->N, desc->K, desc->G, n_pruned, k_per_tile, &sz);
+  if (st != SPG_OK) return st;
+  if (desc->Nk != sz.Nk || desc->T != sz.T || desc->offsetk_len != sz.offsetk_len || ldw < desc->K)
+    return SPG_ERR_INVALID_ARG;
+  if (!desc->offsetn || !desc->tile_n0 || !desc->tile_kofs || !desc->k_per_tile || !desc->offsetk || !desc->Wc)
+    return SPG_ERR_INVALID_ARG;
+  if (ws_bytes < size_t(sz.reorg_ws_bytes)) return SPG_ERR_INVALID_ARG;
+  if (!aligned(W, 2) || !aligned(workspace, 16) || !aligned(desc->Wc, 16)) return SPG_ERR_MISALIGNED;
+  st = check_device();
+  if (st != SPG_OK) return st;
+  const int N = int(sz.N), K = int(sz.K), Nk = int(sz.Nk), T = sz.T;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  // host tables: k per tile and the padded offsets of each tile in offsetk
+  std::vector<int32_t> kofs(T + 1, 0);
+  for (int t = 0; t < T; ++t) kofs[t + 1] = kofs[t] + (k_per_tile[t] + kKBlock - 1) / kKBlock * kKBlock;
+  if (cudaMemcpyAsync(desc->tile_kofs, kofs.data(), sizeof(int32_t) * (T + 1), cudaMemcpyHostToDevice, s) !=
+          cudaSuccess ||
+      cudaMemcpyAsync(desc->k_per_tile, k_per_tile, sizeof(int32_t) * T, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return SPG_ERR_CUDA;
+  auto* keys = static_cast<u128*>(workspace);
+  auto* kept = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + int64_t(N) * 16);
+  const auto* W16 = static_cast<const uint16_t*>(W);
+  col_keys_kernel<<<(N + 7) / 8, 256, 0, s>>>(W16, ldw, N, K, keys);
+  col_prune_kernel<<<(N + 255) / 256, 256, 0, s>>>(keys, N, int(n_pruned), kept);
+  col_compact_kernel<<<1, 1024, 0, s>>>(kept, N, T, desc->offsetn, desc->tile_n0);
+  const int rows_smem = K * (16 + 4);
+  if (cudaFuncSetAttribute(tile_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, rows_smem) != cudaSuccess)
+    return SPG_ERR_CUDA;
+  tile_rows_kernel<<<T, 256, rows_smem, s>>>(W16, ldw, K, Nk, desc->offsetn, desc->tile_kofs, desc->k_per_tile,
+                                             desc->offsetk);
+  int max_blocks = 0;
+  for (int t = 0; t < T; ++t) max_blocks = std::max(max_blocks, (kofs[t + 1] - kofs[t]) / kKBlock);
+  gather_wc_kernel<<<dim3(T, max_blocks), 256, 0, s>>>(W16, ldw, Nk, desc->offsetn, desc->tile_kofs,
+                                                       desc->k_per_tile, desc->offsetk,
+                                                       static_cast<uint16_t*>(desc->Wc));
+  return launch_status();
 }
 
 spg_status spgemm_tw_f16(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Y, int64_t ldy,
                          int64_t M, void* workspace, size_t ws_bytes, spg_stream_t stream) {
-  (void)X; (void)ldx; (void)x_layout; (void)desc; (void)Y; (void)ldy; (void)M; (void)workspace; (void)ws_bytes;
-  (void)stream;
-  return SPG_ERR_UNSUPPORTED_SHAPE;
+  using namespace spg;
+  using namespace spg::tw;
+  if (!X || !desc || !Y) return SPG_ERR_INVALID_ARG;
+  if (x_layout != SPG_X_MK && x_layout != SPG_X_KM) return SPG_ERR_INVALID_ARG;
+  const int64_t N = desc->N, K = desc->K;
+  if (M <= 0 || N <= 0 || K <= 0 || ldy < N) return SPG_ERR_INVALID_ARG;
+  if (desc->G != kG || desc->T <= 0 || desc->offsetk_len <= 0 || desc->offsetk_len % kKBlock) return SPG_ERR_INVALID_ARG;
+  if (!desc->offsetn || !desc->tile_n0 || !desc->tile_kofs || !desc->offsetk || !desc->Wc) return SPG_ERR_INVALID_ARG;
+  if (x_layout == SPG_X_MK ? ldx < K : ldx < M) return SPG_ERR_INVALID_ARG;
+  if (M % 8 || M >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(X, 16) || !aligned(Y, 2) || ldx % 8) return SPG_ERR_MISALIGNED;
+  if (x_layout == SPG_X_MK) {
+    if (!workspace || ws_bytes < tw_workspace_size(M, K, x_layout)) return SPG_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SPG_ERR_MISALIGNED;
+  }
+  spg_status st = check_device();
+  if (st != SPG_OK) return st;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t* xt = static_cast<const uint16_t*>(X);
+  int64_t ldt = ldx;
+  if (x_layout == SPG_X_MK) {
+    uint16_t* ws = static_cast<uint16_t*>(workspace);
+    dim3 grid(static_cast<unsigned>((K + 63) / 64), static_cast<unsigned>((M + 63) / 64));
+    transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(static_cast<const uint16_t*>(X), ldx, int(M), int(K), ws, M);
+    xt = ws;
+    ldt = M;
+  }
+  CUtensorMap tmWc;
+  const uint64_t wc_rows = uint64_t(desc->offsetk_len / kKBlock) * kG;
+  if (!make_tmap_2d(&tmWc, desc->Wc, 2, kKBlock, wc_rows, kKBlock * 2, kKBlock, kG, true)) return SPG_ERR_CUDA;
+  uint32_t* err = device_error_word();
+  if (!err) return SPG_ERR_CUDA;
+  if (cudaFuncSetAttribute(tw_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
+    return SPG_ERR_CUDA;
+  const int64_t units = int64_t(desc->T) * ((M + BN - 1) / BN);
+  const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
+  tw_gemm_kernel<<<grid, 256, SMEM, s>>>(tmWc, xt, ldt, static_cast<uint16_t*>(Y), ldy, int(M), int(desc->Nk),
+                                         desc->T, desc->offsetn, desc->tile_n0, desc->tile_kofs, desc->offsetk,
+                                         err);
+  return launch_status();
 }
 
 }  // extern "C"

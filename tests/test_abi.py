@@ -46,6 +46,7 @@ def test_host_only_calls():
     assert (sz.Nk, sz.T) == (691, 6)
     assert sz.offsetk_len == sum((k + 63) // 64 * 64 for k in (260, 290, 272, 118, 245, 187))
     assert sz.wc_elems == sz.offsetk_len * 128
+    assert sz.reorg_ws_bytes >= 768 * 20
     assert L.tw_query_sizes(768, 768, 64, 77, kpt, ctypes.byref(sz)) == 2      # G must be 128
     assert L.tw_query_sizes(768, 768, 128, 768, kpt, ctypes.byref(sz)) == 1    # n_pruned < N
     assert L.tw_workspace_size(4096, 768, spg.SPG_X_MK) == 4096 * 768 * 2
