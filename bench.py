@@ -44,6 +44,35 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+PROFILED = {  # workload -> (profile summary, kernel sources whose hash it records)
+    "vitb_mlp_f16": ("spgemm24_kernel.vitb_mlp_f16.md", ["spgemm24.cu", "sm100.cuh"]),
+    "tw_bert_f16": ("tw_gemm_kernel.tw_bert_f16.md", ["tw.cu", "sm100.cuh"]),
+}
+
+
+def profiled_traffic(workload):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu summary,
+    or None when there is none or the kernel source changed since it was taken."""
+    import hashlib
+    if workload not in PROFILED:
+        return None
+    md, srcs = PROFILED[workload]
+    path = os.path.join(ROOT, "profiles", md)
+    if not os.path.exists(path):
+        return None
+    want, traffic = None, None
+    for line in open(path):
+        if line.startswith("kernel_source_sha256:"):
+            want = line.split(":", 1)[1].strip()
+        elif line.startswith("dram_bytes_per_launch:"):
+            traffic = int(line.split(":", 1)[1].strip())
+    h = hashlib.sha256()
+    for f in srcs:
+        with open(os.path.join(ROOT, "structured_sparse_gemm_02_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return traffic if want == h.hexdigest()[:16] else None
+
+
 def layer_flops(layers):
     return sum(2.0 * d["M"] * d["N"] * d["K"] for d in layers)
 
@@ -275,7 +304,8 @@ def run_ours(args, rank, world, local_rank):
         per_launch_bytes = bytes_alg / nl
         achieved = per_launch_bytes / (np.mean(lay_ms) * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None, "peak_source": src,
+                "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic(args.workload),
+                "peak_source": src,
                 "kernel": "spgemm24_kernel" if kind != "tw_f16" else "tw_gemm_kernel"}
     else:
         # dense-equivalent FLOPs per launch against the 2:4 sparse tensor peak of the dtype:
@@ -285,7 +315,8 @@ def run_ours(args, rank, world, local_rank):
         per_launch = flops_dense / nl
         achieved = per_launch / (np.mean(lay_ms) * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None, "peak_source": f"{src} bf16 dense x{ratio:g}",
+                "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                "peak_source": f"{src} burst bf16 dense x{ratio:g} (2:4 sparse rate)",
                 "kernel": "spgemm24_kernel"}
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
