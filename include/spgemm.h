@@ -226,6 +226,32 @@ size_t tw_workspace_size(int64_t M, int64_t K, int x_layout);
 spg_status spgemm_tw_f16(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Y,
                          int64_t ldy, int64_t M, void* workspace, size_t ws_bytes, spg_stream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * spgemm_tw_f16_noalloc  (no counterpart on the pages: an interface addition)
+ *
+ * spgemm_tw_f16 with x_layout SPG_X_MK for callers that cannot allocate device
+ * memory themselves -- for instance a plug-in running inside a host framework
+ * that owns every device allocation and forbids extensions from calling
+ * cudaMalloc, or a latency-critical caller that must not pay cudaMalloc's
+ * implicit device synchronisation.  The transposed activations [K][M] are
+ * kept in a fixed 8 MiB device array inside the library instead of a
+ * caller-provided workspace; the caller still passes X, the descriptor and Y.
+ *   Same arguments, limits and results as spgemm_tw_f16(X, ldx, SPG_X_MK, desc,
+ *   Y, ldy, M, ...), and additionally M * K * 2 <= 8 MiB, else
+ *   SPG_ERR_UNSUPPORTED_SHAPE (nothing is launched).
+ *   The array is allocated when the library is loaded and every GPU that
+ *   loads it holds the 8 MiB until the process exits.  No call allocates or
+ *   frees memory.  The first call on a device looks up the array's device
+ *   address once (cudaGetSymbolAddress); make that first call before any
+ *   stream capture.
+ *   All calls share the one array and each call overwrites the part it
+ *   reads, so nothing needs clearing between calls; calls that overlap on the
+ *   GPU (different streams, or different host threads without ordering) race
+ *   on it and must be serialised by the caller.
+ * ------------------------------------------------------------------------- */
+spg_status spgemm_tw_f16_noalloc(const void* X, int64_t ldx, const spg_tw_desc* desc, void* Y, int64_t ldy,
+                                 int64_t M, spg_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

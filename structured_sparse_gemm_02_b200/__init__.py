@@ -54,6 +54,7 @@ SIGNATURES = {
     "tw_workspace_size": (_sz, [_i64, _i64, ctypes.c_int]),
     "spgemm_tw_f16": (ctypes.c_int, [_p, _i64, ctypes.c_int, ctypes.POINTER(SpgTwDesc), _p, _i64, _i64, _p,
                                      _sz, _p]),
+    "spgemm_tw_f16_noalloc": (ctypes.c_int, [_p, _i64, ctypes.POINTER(SpgTwDesc), _p, _i64, _i64, _p]),
 }
 
 _lib = None
@@ -219,4 +220,21 @@ def spgemm_tw_f16(X, desc: TwDesc, x_layout=SPG_X_MK, Y=None, workspace=None, M:
     _check("spgemm_tw_f16", lib().spgemm_tw_f16(
         _ptr(X), X.stride(0), x_layout, ctypes.byref(desc.c), _ptr(Y), Y.stride(0), M, _ptr(workspace),
         ws if workspace is not None else 0, _stream(stream)))
+    return Y
+
+
+def spgemm_tw_f16_noalloc(X, desc: TwDesc, Y=None, stream=None):
+    """Tile-wise GEMM on X [M, K] for callers that cannot allocate device memory.
+
+    The transposed activations live in the library's fixed 8 MiB device array
+    (M * K * 2 bytes at most) instead of a workspace; calls sharing it must not
+    overlap on the GPU.
+    """
+    import torch
+    M = X.shape[0]
+    N = desc.sizes.N
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    _check("spgemm_tw_f16_noalloc", lib().spgemm_tw_f16_noalloc(
+        _ptr(X), X.stride(0), ctypes.byref(desc.c), _ptr(Y), Y.stride(0), M, _stream(stream)))
     return Y

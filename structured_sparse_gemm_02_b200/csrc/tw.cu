@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 #include <vector>
 
 #include "host.cuh"
@@ -517,6 +518,36 @@ spg_status query(int64_t N, int64_t K, int32_t G, int64_t n_pruned, const int32_
   return SPG_OK;
 }
 
+// ---- scratch for the entry point that allocates nothing ------------------------------------
+// spgemm_tw_f16_noalloc keeps the transposed activations [K][M] in this
+// file-scope device array instead of a caller-provided workspace.  Every GPU
+// that loads the library holds it until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB: M*K*2 bytes at most
+static __device__ __align__(256) uint16_t g_noalloc_xt[kNoAllocScratchBytes / 2];
+
+// Device address of g_noalloc_xt on the current device (looked up once per
+// device; the name itself is only a host-side stand-in for the symbol).
+uint16_t* noalloc_scratch(spg_status* st) {
+  static std::mutex mu;
+  static uint16_t* ptr[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    *st = SPG_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_xt) != cudaSuccess || !p) {
+      *st = SPG_ERR_CUDA;
+      return nullptr;
+    }
+    ptr[dev] = static_cast<uint16_t*>(p);
+  }
+  *st = SPG_OK;
+  return ptr[dev];
+}
+
 }  // namespace tw
 }  // namespace spg
 
@@ -617,6 +648,45 @@ spg_status spgemm_tw_f16(const void* X, int64_t ldx, int x_layout, const spg_tw_
   tw_gemm_kernel<<<grid, 256, SMEM, s>>>(tmWc, xt, ldt, static_cast<uint16_t*>(Y), ldy, int(M), int(desc->Nk),
                                          desc->T, desc->offsetn, desc->tile_n0, desc->tile_kofs, desc->offsetk,
                                          err);
+  return launch_status();
+}
+
+// Tile-wise GEMM on [M, K] activations for callers that cannot allocate
+// device memory: the transposed activations go to the library's own 8 MiB
+// device array instead of a caller workspace.  Same results as
+// spgemm_tw_f16(..., SPG_X_MK, ...).
+spg_status spgemm_tw_f16_noalloc(const void* X, int64_t ldx, const spg_tw_desc* desc, void* Y, int64_t ldy,
+                                 int64_t M, spg_stream_t stream) {
+  using namespace spg;
+  using namespace spg::tw;
+  if (!X || !desc || !Y) return SPG_ERR_INVALID_ARG;
+  const int64_t N = desc->N, K = desc->K;
+  if (M <= 0 || N <= 0 || K <= 0 || ldy < N || ldx < K) return SPG_ERR_INVALID_ARG;
+  if (desc->G != kG || desc->T <= 0 || desc->offsetk_len <= 0 || desc->offsetk_len % kKBlock) return SPG_ERR_INVALID_ARG;
+  if (!desc->offsetn || !desc->tile_n0 || !desc->tile_kofs || !desc->offsetk || !desc->Wc) return SPG_ERR_INVALID_ARG;
+  if (M % 8 || M >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
+  if (uint64_t(M) * uint64_t(K) * 2u > kNoAllocScratchBytes) return SPG_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(X, 16) || !aligned(Y, 2) || ldx % 8) return SPG_ERR_MISALIGNED;
+  spg_status st = check_device();
+  if (st != SPG_OK) return st;
+  uint16_t* xt = noalloc_scratch(&st);
+  if (st != SPG_OK) return st;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  // every element of the [K][M] region the GEMM reads is written here first,
+  // so nothing left in the array by an earlier call is ever read
+  dim3 tgrid(static_cast<unsigned>((K + 63) / 64), static_cast<unsigned>((M + 63) / 64));
+  transpose_kernel<<<tgrid, dim3(32, 8), 0, s>>>(static_cast<const uint16_t*>(X), ldx, int(M), int(K), xt, M);
+  CUtensorMap tmWc;
+  const uint64_t wc_rows = uint64_t(desc->offsetk_len / kKBlock) * kG;
+  if (!make_tmap_2d(&tmWc, desc->Wc, 2, kKBlock, wc_rows, kKBlock * 2, kKBlock, kG, true)) return SPG_ERR_CUDA;
+  uint32_t* err = device_error_word();
+  if (!err) return SPG_ERR_CUDA;
+  if (cudaFuncSetAttribute(tw_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
+    return SPG_ERR_CUDA;
+  const int64_t units = int64_t(desc->T) * ((M + BN - 1) / BN);
+  const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
+  tw_gemm_kernel<<<grid, 256, SMEM, s>>>(tmWc, xt, M, static_cast<uint16_t*>(Y), ldy, int(M), int(desc->Nk), desc->T,
+                                         desc->offsetn, desc->tile_n0, desc->tile_kofs, desc->offsetk, err);
   return launch_status();
 }
 
