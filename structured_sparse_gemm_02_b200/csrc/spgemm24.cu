@@ -414,7 +414,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     for (int t = pair; t < total; t += npairs, ++i) {
       const int n0 = (t % NT) * 256 + 128 * int(rank), m0 = (t / NT) * BN;
       const int b = i & 1;
-      if (!mbar_wait_warp(&acc_full[b], (i >> 1) & 1, abort_flag, err, ERR_WAIT_ACC)) break;
+      // the two warps of a pair take the same branch: they meet at the pair barrier below
+      const bool got = mbar_wait_warp(&acc_full[b], (i >> 1) & 1, abort_flag, err, ERR_WAIT_ACC);
+      if (!named_bar_all(pair_bar, 64, got)) break;
       tc_fence_after();
       const int nb = n0 + 32 * q;
       const int n = nb + lane;

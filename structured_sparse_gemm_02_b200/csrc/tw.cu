@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 #include <vector>
 
@@ -215,23 +216,44 @@ __global__ void transpose_kernel(const uint16_t* __restrict__ X, int64_t ldx, in
 }
 
 // ---- run-time GEMM -------------------------------------------------------------------------
+// ---- run-time GEMM -------------------------------------------------------------------------
 // Work unit (tile t, 128-row block of X): D[j][m] = sum_i Wc_t[j][i] * X[m][offsetk_t[i]]
 // on the dense tensor cores (A = condensed tile, K-major; B = gathered rows of
 // Xt, MN-major), then Y[m][offsetn[tG+j]] = D[j][m] and +0 in the tile's
-// pruned columns.  Persistent CTAs, warp 0 loads (TMA for the tile block,
-// 16-byte cp.async per lane for the kept rows of Xt), warp 2 issues
-// tcgen05.mma into one of two accumulators, warps 4-7 drain, stage the
-// tile's output span in shared memory and write whole rows of Y.
+// pruned columns.  Persistent CTAs with warp roles (384 threads):
+//   warps 0-1  loads: warp 0 lane 0 issues the TMA of the condensed tile
+//              block; each lane of both warps gathers kept rows of Xt with
+//              16-byte cp.async (warp w takes rows 32w..32w+31 of a block).
+//              The 64 row indices of a block are read one block ahead, and
+//              the scalars of the next unit one unit ahead, so no copy waits
+//              on a dependent index load.
+//   warp 2     TMEM owner and MMA issuer (two accumulators)
+//   warps 4-11 drain, in two groups of four warps that each own 64 rows of
+//              the unit: tcgen05.ld of the accumulator (released at once).  The
+//              16-byte-aligned middle of the unit's output span
+//              [tile_n0[t], tile_n0[t+1]) is assembled in double-buffered
+//              shared memory, 184 columns at a time (zeroed, then each lane
+//              places its kept column), and leaves as a few 2-D TMA stores;
+//              the ragged ends (at most 7 columns a side) are assembled the
+//              same way in a [128][16] edge buffer and leave with one store
+//              instruction per row for both ends.
 constexpr int BN = 128;                   // X rows per work unit
 constexpr int A_BYTES = kG * kKBlock * 2;  // 16 KB
 constexpr int B_BYTES = kKBlock * BN * 2;  // 16 KB: 64 gathered rows x 128 m, two 64-wide atoms
 constexpr int STAGES = 4;
-constexpr int MAX_SPAN = 256;              // widest tile output span staged in shared memory
+constexpr int EPI_GROUPS = 2;              // drain groups of 4 warps, each owning RG rows of a unit
+constexpr int RG = BN / EPI_GROUPS;        // 64
+constexpr int THREADS = 128 + 128 * EPI_GROUPS;
+constexpr int WIN = 184;                   // output columns staged per window (a multiple of 8)
+constexpr int WIN_ELEMS = RG * WIN;        // one staging buffer: [64 rows] x WIN, box-blocked
 constexpr int OFF_STG = STAGES * (A_BYTES + B_BYTES);
-constexpr int OFF_BAR = OFF_STG + BN * MAX_SPAN * 2;
+constexpr int OFF_EDGE = OFF_STG + EPI_GROUPS * 2 * WIN_ELEMS * 2;  // two staging buffers per group
+constexpr int OFF_BAR = OFF_EDGE + EPI_GROUPS * RG * 16 * 2;
 constexpr int SMEM = OFF_BAR + (2 * STAGES + 5) * 8 + 16 + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
+static_assert(WIN % 8 == 0 && (WIN_ELEMS * 2) % 1024 == 0 && OFF_STG % 1024 == 0, "staging blocks stay aligned");
 constexpr uint32_t TMEM_COLS = 256;
+constexpr int kLoadLanes = 64;             // cp.async arrivals per stage (two gather warps)
 
 __device__ __forceinline__ void tail_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
   int never = 0;
@@ -250,9 +272,11 @@ __device__ __forceinline__ void cp_async_arrive(uint64_t* bar) {
 
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-__global__ void __launch_bounds__(256, 1)
-    tw_gemm_kernel(const __grid_constant__ CUtensorMap tmWc, const uint16_t* __restrict__ xt, int64_t ldt,
-                   uint16_t* __restrict__ Y, int64_t ldy, int M, int Nk, int T, const int* __restrict__ offsetn,
+__global__ void __launch_bounds__(THREADS, 1)
+    tw_gemm_kernel(const __grid_constant__ CUtensorMap tmWc, const __grid_constant__ CUtensorMap tmY64,
+                   const __grid_constant__ CUtensorMap tmY8, const uint16_t* __restrict__ xt, int64_t ldt,
+                   uint16_t* __restrict__ Y, int64_t ldy, int vec_ok, int M, int Nk, int T,
+                   const int* __restrict__ offsetn,
                    const int* __restrict__ tile_n0, const int* __restrict__ tile_kofs,
                    const int* __restrict__ offsetk, uint32_t* err) {
   extern __shared__ uint8_t smem_raw[];
@@ -271,18 +295,24 @@ __global__ void __launch_bounds__(256, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 33);  // TMA of the tile block + one cp.async arrival per producer lane
+      mbar_init(&full[s], 1 + kLoadLanes);  // TMA of the tile block + one cp.async arrival per gather lane
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);
+      mbar_init(&acc_empty[b], 4 * EPI_GROUPS);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmWc);
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmWc);
+    if (vec_ok) {
+      tma_prefetch_desc(&tmY64);
+      tma_prefetch_desc(&tmY8);
+    }
+  }
   if (warp == 2) {
     tmem_alloc(tmem_holder, TMEM_COLS);
     tmem_relinquish();
@@ -292,67 +322,70 @@ __global__ void __launch_bounds__(256, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
-  if (warp == 0) {
+  if (warp < 2) {
     // ---------------- loads ----------------
-    // The 64 row indices of a K block are read by the whole warp (two per
-    // lane) one block ahead of their use; lane 0 issues the copies.
     uint32_t g = 0;
     bool ok = true;
+    const int rbase = 32 * warp;  // this warp's rows within a block
+    const int a = (lane >> 3) & 1, c = lane & 7, hl = lane >> 4;
     int u = blockIdx.x;
-    int kb = 0;
-    // indices of the next block to issue
-    int nxt0 = 0, nxt1 = 0;
-    auto load_idx = [&](int uu, int kk) {
-      if (uu < units) {
-        const int* rows = offsetk + tile_kofs[uu / MB] + kk * kKBlock;
-        nxt0 = rows[lane];
-        nxt1 = rows[32 + lane];
-      }
-    };
-    load_idx(u, 0);
+    // scalars of the current unit, and the first row indices of its block 0
+    int kofs = 0, KB = 0, nxt = 0;
+    if (u < units) {
+      const int t = u / MB;
+      kofs = tile_kofs[t];
+      KB = (tile_kofs[t + 1] - kofs) / kKBlock;
+      nxt = offsetk[kofs + rbase + lane];
+    }
     while (ok && u < units) {
-      const int t = u / MB, mb = (u % MB) * BN;
-      const int kofs = tile_kofs[t];
-      const int KB = (tile_kofs[t + 1] - kofs) / kKBlock;
-      const int cur0 = nxt0, cur1 = nxt1;
-      // advance to the following block and prefetch its indices
-      int un = u, kn = kb + 1;
-      if (kn == KB) {
-        un = u + gridDim.x;
-        kn = 0;
-      }
-      load_idx(un, kn);
-      const int s = g % STAGES;
-      const uint32_t use = g / STAGES;
-      if (use > 0 && !mbar_wait_warp(&empty[s], (use - 1) & 1, abort_flag, err, ERR_WAIT_EMPTY)) {
-        ok = false;
-        break;
-      }
-      uint8_t* a_s = smem + s * (A_BYTES + B_BYTES);
-      const uint32_t b_s = smem_addr(a_s + A_BYTES);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&full[s], A_BYTES);
-        tma_load_2d(a_s, &tmWc, 0, (kofs / kKBlock + kb) * kG, &full[s]);
-      }
-      // B: the 64 kept rows of Xt for this block, 128 m each, as two MN-major
-      // 128-byte-swizzled atoms of 64 m (chunk c of row r at chunk c ^ (r % 8))
-      const int a = (lane >> 3) & 1, c = lane & 7;
+      const int mb = (u % MB) * BN;
       const int mcol = mb + 64 * a + 8 * c;
       const uint32_t src_bytes = mcol < M ? 16u : 0u;
-#pragma unroll
-      for (int i = 0; i < kKBlock / 2; ++i) {
-        const int r = 2 * i + (lane >> 4);
-        const int rk = __shfl_sync(0xffffffffu, i < 16 ? cur0 : cur1, r & 31);
-        const uint32_t dst = b_s + a * 8192 + r * 128 + ((c ^ (r & 7)) << 4);
-        cp_async16(dst, xt + int64_t(rk) * ldt + (src_bytes ? mcol : 0), src_bytes);
+      const uint16_t* xcol = xt + (src_bytes ? mcol : 0);
+      // scalars of the next unit, loaded while this one is issued
+      const int un = u + gridDim.x;
+      int kofs_n = 0, KB_n = 0;
+      if (un < units) {
+        const int tn = un / MB;
+        kofs_n = tile_kofs[tn];
+        KB_n = (tile_kofs[tn + 1] - kofs_n) / kKBlock;
       }
-      cp_async_arrive(&full[s]);
-      ++g;
+      for (int kb = 0; kb < KB; ++kb, ++g) {
+        const int cur = nxt;
+        if (kb + 1 < KB)
+          nxt = offsetk[kofs + (kb + 1) * kKBlock + rbase + lane];
+        else if (un < units)
+          nxt = offsetk[kofs_n + rbase + lane];
+        const int s = g % STAGES;
+        const uint32_t use = g / STAGES;
+        if (use > 0 && !mbar_wait_warp(&empty[s], (use - 1) & 1, abort_flag, err, ERR_WAIT_EMPTY)) {
+          ok = false;
+          break;
+        }
+        uint8_t* a_s = smem + s * (A_BYTES + B_BYTES);
+        const uint32_t b_s = smem_addr(a_s + A_BYTES);
+        if (warp == 0 && lane == 0) {
+          mbar_arrive_expect_tx(&full[s], A_BYTES);
+          tma_load_2d(a_s, &tmWc, 0, (kofs / kKBlock + kb) * kG, &full[s]);
+        }
+        // B: kept rows of Xt, 128 m each, as two MN-major 128-byte-swizzled
+        // atoms of 64 m (16-byte chunk c of row r at chunk c ^ (r % 8))
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int rl = 2 * i + hl;
+          const int r = rbase + rl;
+          const int rk = __shfl_sync(0xffffffffu, cur, rl);
+          const uint32_t dst = b_s + a * 8192 + r * 128 + ((c ^ (r & 7)) << 4);
+          cp_async16(dst, xcol + int64_t(rk) * ldt, src_bytes);
+        }
+        cp_async_arrive(&full[s]);
+      }
       u = un;
-      kb = kn;
+      kofs = kofs_n;
+      KB = KB_n;
     }
     cp_async_wait_all();
-    if (lane == 0)
+    if (warp == 0 && lane == 0)
       for (uint32_t q = (g > uint32_t(STAGES) ? g - STAGES : 0u); q < g; ++q)
         tail_wait(&full[q % STAGES], (q / STAGES) & 1, err);
     __syncwarp();
@@ -402,84 +435,137 @@ __global__ void __launch_bounds__(256, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ---------------- drain and scatter ----------------
+    // Group eg (warps 4-7: eg 0, warps 8-11: eg 1) drains rows [64 eg, 64 eg + 64)
+    // of every unit: TMEM columns b*BN + 64 eg .. +63 of the lanes of quadrant q.
     const int q = warp & 3;
+    const int eg = (warp - 4) >> 2;
+    const int gtid = threadIdx.x - 128 - 128 * eg;  // 0..127 within the group
+    const uint32_t bar_win = 1 + eg, bar_vote = 3 + eg;
+    uint16_t* stg0 = reinterpret_cast<uint16_t*>(smem + OFF_STG + eg * (2 * WIN_ELEMS * 2));
+    uint16_t* edge = reinterpret_cast<uint16_t*>(smem + OFF_EDGE + eg * (RG * 16 * 2));  // [64 rows][16]
+    uint32_t wc = 0;  // windows staged so far: window w uses staging buffer w % 2
     int i = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++i) {
-      const int t = u / MB, mb = (u % MB) * BN;
+      const int t = u / MB;
+      const int mb = (u % MB) * BN + RG * eg;  // first row of this group
       const int b = i & 1;
-      if (!mbar_wait_warp(&acc_full[b], (i >> 1) & 1, abort_flag, err, ERR_WAIT_ACC)) break;
-      tc_fence_after();
-      uint32_t r[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld_32x32b_x32(tmem + (uint32_t(32 * q) << 16) + uint32_t(b * BN + 32 * c), r[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acc_empty[b]);
-
+      // tile scalars first: their loads overlap the wait for the accumulator
       const int j0 = t * kG;
       const int Gt = min(kG, Nk - j0);
       const int j = 32 * q + lane;
       const bool valid = j < Gt;
       const int nj = valid ? offsetn[j0 + j] : 0;
       const int n0 = tile_n0[t], n1 = tile_n0[t + 1];
-      const int span = n1 - n0;
-      // pruned columns owned by this lane: the gap after its kept column, and
-      // for the first kept column of the tile also the gap before it
-      const int gap_end = valid ? (j + 1 < Gt ? offsetn[j0 + j + 1] : n1) : 0;
-      const int lead0 = (valid && j == 0) ? n0 : 0;
-      const int lead1 = (valid && j == 0) ? nj : 0;
-      const int rows = min(BN, M - mb);
-      if (span <= MAX_SPAN) {
-        // stage the output rows of the span (kept values and zeros) and write
-        // every row of Y contiguously
-        uint16_t* stg = reinterpret_cast<uint16_t*>(smem + OFF_STG);
-        named_bar_sync(1, 128);  // the previous unit's rows have been written out
-        if (valid) {
-          const int col = nj - n0;
+      const int rows = max(0, min(RG, M - mb));
+      // Columns [s0, s1) are staged in windows; with 16-byte rows that is the
+      // aligned middle of the span (TMA stores) and the ragged ends [n0, a0),
+      // [a1, n1) go through the edge buffer; otherwise every column of the
+      // span is staged and copied out by element stores.
+      int s0, s1, a0 = n0, a1 = n1;
+      if (vec_ok) {
+        a0 = (n0 + 7) & ~7;
+        a1 = max(a0, n1 & ~7);
+        s0 = a0;
+        s1 = a1;
+      } else {
+        s0 = n0 & ~7;
+        s1 = (n1 + 7) & ~7;
+      }
+      const int e1 = n0 & ~7;  // edge slots 0-7: columns [e1, e1 + 8); slots 8-15: [a1, a1 + 8)
+      // the four warps of the group take the same branch: they meet at named barriers below
+      const bool got = mbar_wait_warp(&acc_full[b], (i >> 1) & 1, abort_flag, err, ERR_WAIT_ACC);
+      if (!named_bar_all(bar_vote, 128, got)) break;
+      tc_fence_after();
+      uint32_t r[2][32];
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
+      for (int cc = 0; cc < 2; ++cc)
+        tmem_ld_32x32b_x32(tmem + (uint32_t(32 * q) << 16) + uint32_t(b * BN + RG * eg + 32 * cc), r[cc]);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
+
+      // Windows: zero, place kept columns, store.  Layout of a window of ww
+      // columns (a multiple of 8): nw blocks [64 rows][64 columns] then nn
+      // blocks [64 rows][8 columns], the shapes of the two TMA store boxes.
+      // The first pass also zeroes and fills the edge buffer (even with no window).
+      for (int x0 = s0, pass = 0; pass == 0 || x0 < s1; x0 += WIN, ++pass) {
+        const int ww = max(0, min(WIN, s1 - x0));
+        const int nw = ww >> 6, nn = (ww & 63) >> 3;
+        uint16_t* stg = stg0 + (wc & 1) * WIN_ELEMS;
+        {
+          uint4* z = reinterpret_cast<uint4*>(stg);
+          const int nz = ww * (RG / 8);
+          for (int e = gtid; e < nz; e += 128) z[e] = make_uint4(0u, 0u, 0u, 0u);
+          if (pass == 0 && gtid < RG * 2) reinterpret_cast<uint4*>(edge)[gtid] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        named_bar_sync(bar_win, 128);
+        int off = -1, rs = 0;
+        if (valid && nj >= x0 && nj < x0 + ww) {
+          const int rel = nj - x0;
+          if (rel < 64 * nw) {
+            off = (rel >> 6) * (RG * 64) + (rel & 63);
+            rs = 64;
+          } else {
+            const int r2 = rel - 64 * nw;
+            off = nw * (RG * 64) + (r2 >> 3) * (RG * 8) + (r2 & 7);
+            rs = 8;
+          }
+        }
+        uint16_t* dst = stg + off;
+        if (pass == 0 && vec_ok && valid && (nj < a0 || nj >= a1)) {
+          dst = edge + (nj < a0 ? nj - e1 : 8 + nj - a1);
+          rs = 16;
+          off = 0;
+        }
+        if (off >= 0) {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
             for (int k = 0; k < 32; ++k)
-              stg[(32 * cc + k) * MAX_SPAN + col] = __half_as_ushort(__float2half_rn(__uint_as_float(r[cc][k])));
-          if (gap_end > nj + 1 || lead1 > lead0) {
-#pragma unroll 1
-            for (int k = 0; k < BN; ++k) {
-              for (int z = nj + 1; z < gap_end; ++z) stg[k * MAX_SPAN + z - n0] = 0;
-              for (int z = lead0; z < lead1; ++z) stg[k * MAX_SPAN + z - n0] = 0;
+              dst[(32 * cc + k) * rs] = __half_as_ushort(__float2half_rn(__uint_as_float(r[cc][k])));
+        }
+        fence_proxy_async_smem();             // staged rows -> the TMA stores below
+        if (gtid == 0) bulk_wait_read<0>();   // the previous window's stores have read their buffer
+        named_bar_sync(bar_win, 128);
+        if (ww > 0) {
+          if (vec_ok) {
+            if (gtid == 0 && rows > 0) {
+              const uint32_t sb = smem_addr(stg);
+              for (int g = 0; g < nw; ++g)
+                tma_store_2d_saddr(&tmY64, sb + uint32_t(g * RG * 64 * 2), x0 + 64 * g, mb);
+              for (int h = 0; h < nn; ++h)
+                tma_store_2d_saddr(&tmY8, sb + uint32_t((nw * RG * 64 + h * RG * 8) * 2), x0 + 64 * nw + 8 * h,
+                                   mb);
+              bulk_commit();
             }
+          } else {
+            // element stores, lanes across the columns of a row
+            for (int row = q; row < rows; row += 4) {
+              uint16_t* yrow = Y + int64_t(mb + row) * ldy;
+              for (int rel = lane; rel < ww; rel += 32) {
+                const int col = x0 + rel;
+                const int so = rel < 64 * nw ? (rel >> 6) * (RG * 64) + row * 64 + (rel & 63)
+                                             : nw * (RG * 64) + ((rel - 64 * nw) >> 3) * (RG * 8) + row * 8 +
+                                                   ((rel - 64 * nw) & 7);
+                if (col >= n0 && col < n1) yrow[col] = stg[so];
+              }
+            }
+            named_bar_sync(bar_win, 128);  // the buffer is read before it is zeroed again
           }
-        }
-        named_bar_sync(1, 128);
-#pragma unroll 1
-        for (int k = q * 32; k < q * 32 + 32; ++k) {
-          if (k >= rows) break;
-          uint16_t* yrow = Y + int64_t(mb + k) * ldy + n0;
-          const uint16_t* srow = stg + k * MAX_SPAN;
-          for (int cidx = lane; cidx < span; cidx += 32) yrow[cidx] = srow[cidx];
-        }
-      } else {
-        // very wide span: direct stores
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            const int m = mb + 32 * cc + k;
-            if (valid && m < M)
-              Y[int64_t(m) * ldy + nj] = __half_as_ushort(__float2half_rn(__uint_as_float(r[cc][k])));
-          }
-        }
-        if (valid && (gap_end > nj + 1 || lead1 > lead0)) {
-#pragma unroll 1
-          for (int k = 0; k < rows; ++k) {
-            uint16_t* yrow = Y + int64_t(mb + k) * ldy;
-            for (int z = nj + 1; z < gap_end; ++z) yrow[z] = 0;
-            for (int z = lead0; z < lead1; ++z) yrow[z] = 0;
-          }
+          ++wc;
         }
       }
+      // ragged ends (16-byte rows only): one instruction per row covers both
+      // edge sectors; lanes 0-7 the head chunk, lanes 8-15 the tail chunk
+      if (vec_ok && (n0 < a0 || a1 < n1) && lane < 16) {
+        const int col = lane < 8 ? e1 + lane : a1 + lane - 8;
+        const bool mine = lane < 8 ? (col >= n0 && col < a0 && col < n1) : (col < n1);
+        if (mine)
+          for (int row = q; row < rows; row += 4) Y[int64_t(mb + row) * ldy + col] = edge[row * 16 + lane];
+      }
     }
+    if (gtid == 0) bulk_wait_all<0>();
   }
 
   tc_fence_before();
@@ -491,9 +577,27 @@ __global__ void __launch_bounds__(256, 1)
 }
 
 int sm_count() {
-  int dev = 0, v = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-  return v;
+  static int cached[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int v = 148;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    cached[dev] = v;
+  }
+  return cached[dev];
+}
+
+// The GEMM's dynamic shared-memory limit, raised once per device.
+bool smem_attr_set() {
+  static int done[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (__atomic_load_n(&done[dev], __ATOMIC_ACQUIRE)) return true;
+  if (cudaFuncSetAttribute(tw_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
+    return false;
+  __atomic_store_n(&done[dev], 1, __ATOMIC_RELEASE);
+  return true;
 }
 
 spg_status query(int64_t N, int64_t K, int32_t G, int64_t n_pruned, const int32_t* kpt, spg_tw_sizes* out) {
@@ -516,6 +620,33 @@ spg_status query(int64_t N, int64_t K, int32_t G, int64_t n_pruned, const int32_
   out->wc_elems = kofs * G;
   out->reorg_ws_bytes = (N * 16 + N * 4 + 255) / 256 * 256;
   return SPG_OK;
+}
+
+// Tensor maps and launch of the run-time GEMM over transposed activations
+// xt [K][ldt] (shared by the entry points below).
+spg_status launch_gemm(const uint16_t* xt, int64_t ldt, const spg_tw_desc* desc, uint16_t* Y, int64_t ldy,
+                       int64_t M, cudaStream_t s) {
+  CUtensorMap tmWc, tmY64, tmY8;
+  const uint64_t wc_rows = uint64_t(desc->offsetk_len / kKBlock) * kG;
+  if (!make_tmap_2d(&tmWc, desc->Wc, 2, kKBlock, wc_rows, kKBlock * 2, kKBlock, kG, true)) return SPG_ERR_CUDA;
+  // Y leaves through TMA when its rows are 16-byte aligned; otherwise by element stores only
+  const int vec_ok = aligned(Y, 16) && (ldy % 8) == 0;
+  if (vec_ok) {
+    if (!make_tmap_2d(&tmY64, Y, 2, uint64_t(desc->N), uint64_t(M), uint64_t(ldy) * 2, 64, RG, false) ||
+        !make_tmap_2d(&tmY8, Y, 2, uint64_t(desc->N), uint64_t(M), uint64_t(ldy) * 2, 8, RG, false))
+      return SPG_ERR_CUDA;
+  } else {
+    std::memset(&tmY64, 0, sizeof(tmY64));
+    std::memset(&tmY8, 0, sizeof(tmY8));
+  }
+  uint32_t* err = device_error_word();
+  if (!err) return SPG_ERR_CUDA;
+  if (!smem_attr_set()) return SPG_ERR_CUDA;
+  const int64_t units = int64_t(desc->T) * ((M + BN - 1) / BN);
+  const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
+  tw_gemm_kernel<<<grid, THREADS, SMEM, s>>>(tmWc, tmY64, tmY8, xt, ldt, Y, ldy, vec_ok, int(M), int(desc->Nk), desc->T,
+                                         desc->offsetn, desc->tile_n0, desc->tile_kofs, desc->offsetk, err);
+  return launch_status();
 }
 
 // ---- scratch for the entry point that allocates nothing ------------------------------------
@@ -636,19 +767,7 @@ spg_status spgemm_tw_f16(const void* X, int64_t ldx, int x_layout, const spg_tw_
     xt = ws;
     ldt = M;
   }
-  CUtensorMap tmWc;
-  const uint64_t wc_rows = uint64_t(desc->offsetk_len / kKBlock) * kG;
-  if (!make_tmap_2d(&tmWc, desc->Wc, 2, kKBlock, wc_rows, kKBlock * 2, kKBlock, kG, true)) return SPG_ERR_CUDA;
-  uint32_t* err = device_error_word();
-  if (!err) return SPG_ERR_CUDA;
-  if (cudaFuncSetAttribute(tw_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
-    return SPG_ERR_CUDA;
-  const int64_t units = int64_t(desc->T) * ((M + BN - 1) / BN);
-  const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
-  tw_gemm_kernel<<<grid, 256, SMEM, s>>>(tmWc, xt, ldt, static_cast<uint16_t*>(Y), ldy, int(M), int(desc->Nk),
-                                         desc->T, desc->offsetn, desc->tile_n0, desc->tile_kofs, desc->offsetk,
-                                         err);
-  return launch_status();
+  return launch_gemm(xt, ldt, desc, static_cast<uint16_t*>(Y), ldy, M, s);
 }
 
 // Tile-wise GEMM on [M, K] activations for callers that cannot allocate
@@ -676,18 +795,7 @@ spg_status spgemm_tw_f16_noalloc(const void* X, int64_t ldx, const spg_tw_desc* 
   // so nothing left in the array by an earlier call is ever read
   dim3 tgrid(static_cast<unsigned>((K + 63) / 64), static_cast<unsigned>((M + 63) / 64));
   transpose_kernel<<<tgrid, dim3(32, 8), 0, s>>>(static_cast<const uint16_t*>(X), ldx, int(M), int(K), xt, M);
-  CUtensorMap tmWc;
-  const uint64_t wc_rows = uint64_t(desc->offsetk_len / kKBlock) * kG;
-  if (!make_tmap_2d(&tmWc, desc->Wc, 2, kKBlock, wc_rows, kKBlock * 2, kKBlock, kG, true)) return SPG_ERR_CUDA;
-  uint32_t* err = device_error_word();
-  if (!err) return SPG_ERR_CUDA;
-  if (cudaFuncSetAttribute(tw_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM) != cudaSuccess)
-    return SPG_ERR_CUDA;
-  const int64_t units = int64_t(desc->T) * ((M + BN - 1) / BN);
-  const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
-  tw_gemm_kernel<<<grid, 256, SMEM, s>>>(tmWc, xt, M, static_cast<uint16_t*>(Y), ldy, int(M), int(desc->Nk), desc->T,
-                                         desc->offsetn, desc->tile_n0, desc->tile_kofs, desc->offsetk, err);
-  return launch_status();
+  return launch_gemm(xt, M, desc, static_cast<uint16_t*>(Y), ldy, M, s);
 }
 
 }  // extern "C"

@@ -135,3 +135,56 @@ def test_bert_layers_parity(spg, layout):
         assert rep["ok"], rep
         pruned = sorted(set(range(d["N"])) - set(r["offsetn"]))
         assert not Y[:, pruned].view(np.uint16).any()   # pruned columns are +0
+
+
+@pytest.mark.parametrize("ldy_pad", [0, 8, 3])
+def test_wide_span_windows_and_pitch(spg, ldy_pad):
+    """A tile owning hundreds of pruned columns (output span wider than one
+    staging window), written through padded row pitches: 16-byte stores when
+    the pitch allows them, element stores otherwise; padding stays untouched."""
+    import torch
+    rng = np.random.default_rng(11)
+    N, K, P, M = 640, 128, 320, 200
+    W = rng.standard_normal((N, K)).astype(np.float16)
+    W[:P] = (W[:P].astype(np.float32) * 1e-3).astype(np.float16)   # the first P columns are pruned first
+    kpt = rng.integers(1, K + 1, (N - P + 127) // 128)
+    X = rng.standard_normal((M, K)).astype(np.float16)
+    desc = spg.tw_reorganize(torch.from_numpy(W).cuda(), 128, P, kpt)
+    ref = tw.tw_reorganize(W, 128, P, kpt)
+    assert ref["tiles"][0]["n1"] - ref["tiles"][0]["n0"] > 256
+    ldy = N + ldy_pad
+    raw = torch.full((M, ldy), 0x7E01, dtype=torch.int16, device="cuda")
+    Y = raw.view(torch.float16)[:, :N]
+    for layout in (spg.SPG_X_MK, spg.SPG_X_KM):
+        Xd = torch.from_numpy(X).cuda()
+        if layout == spg.SPG_X_KM:
+            Xd = Xd.t().contiguous()
+        spg.spgemm_tw_f16(Xd, desc, layout, Y=Y, M=M)
+        assert spg.check_device_error() == 0
+        got = raw.cpu().numpy().view(np.uint16)
+        assert (got[:, N:] == 0x7E01).all()
+        rep = compare.check_close(got[:, :N].view(np.float16).astype(np.float64), tw.tw_gemm_ref(X, ref), K)
+        assert rep["ok"], rep
+        pruned = sorted(set(range(N)) - set(ref["offsetn"]))
+        assert not got[:, pruned].any()
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_short_last_tile_aligned_pitch(spg, seed):
+    """A last tile of 3 kept columns whose span is shorter than one 16-byte
+    chunk, on a pitch that allows TMA stores (both ragged ends in one chunk)."""
+    import torch
+    rng = np.random.default_rng(100 + seed)
+    N, K, P, M = 264, 128, 5, 136
+    W = rng.standard_normal((N, K)).astype(np.float16)
+    kpt = rng.integers(1, K + 1, (N - P + 127) // 128)
+    X = rng.standard_normal((M, K)).astype(np.float16)
+    desc = spg.tw_reorganize(torch.from_numpy(W).cuda(), 128, P, kpt)
+    ref = tw.tw_reorganize(W, 128, P, kpt)
+    assert ref["tiles"][-1]["n1"] - ref["tiles"][-1]["n0"] < 16
+    for layout in (spg.SPG_X_MK, spg.SPG_X_KM):
+        Y = _run_gemm(spg, X, desc, layout, N)
+        rep = compare.check_close(Y.astype(np.float64), tw.tw_gemm_ref(X, ref), K)
+        assert rep["ok"], rep
+        pruned = sorted(set(range(N)) - set(ref["offsetn"]))
+        assert not Y[:, pruned].view(np.uint16).any()
