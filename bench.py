@@ -156,9 +156,9 @@ class Layer24:
     """Device-resident buffers of one 2:4 layer: `copies` rotating sets of X,
     compressed W, metadata, bias and Y."""
 
-    def __init__(self, spg, d, kind, copies):
+    def __init__(self, spg, d, kind, copies, y_nm=False):
         import torch
-        self.spg, self.d, self.kind = spg, d, kind
+        self.spg, self.d, self.kind, self.y_nm = spg, d, kind, y_nm
         dev = torch.device("cuda")
         if kind == "24_s8":
             W = torch.from_numpy(d["W"]).to(dev)
@@ -178,7 +178,8 @@ class Layer24:
         self.Wv = [Wv] + [Wv.clone() for _ in range(copies - 1)]
         self.meta = [meta] + [meta.clone() for _ in range(copies - 1)]
         self.bias = [bias] + [bias.clone() if bias is not None else None for _ in range(copies - 1)]
-        self.Y = [torch.empty((d["M"], d["N"]), dtype=self.out_dtype, device=dev) for _ in range(copies)]
+        yshape = (d["N"], d["M"]) if y_nm else (d["M"], d["N"])
+        self.Y = [torch.empty(yshape, dtype=self.out_dtype, device=dev) for _ in range(copies)]
 
     @staticmethod
     def _t(a, tdt, dev):
@@ -194,14 +195,16 @@ class Layer24:
         Y = self.Y[i] if Y is None else Y
         if self.kind == "24_s8":
             self.spg.spgemm_24_s8(X, self.Wv[i], self.meta[i], self.scale, self.bias[i], Y=Y)
+        elif self.y_nm:
+            self.spg.spgemm_24_f16_yt(X, self.Wv[i], self.meta[i], self.bias[i], Yt=Y)
         else:
             self.spg.spgemm_24_f16(X, self.Wv[i], self.meta[i], self.bias[i], Y=Y)
 
 
 class LayerTW:
-    def __init__(self, spg, d, copies, x_layout):
+    def __init__(self, spg, d, copies, x_layout, y_nm=False):
         import torch
-        self.spg, self.d = spg, d
+        self.spg, self.d, self.y_nm = spg, d, y_nm
         dev = torch.device("cuda")
         W = torch.from_numpy(d["W"]).to(dev)
         self.desc = spg.tw_reorganize(W, d["G"], d["n_pruned"], list(d["k_per_tile"]))
@@ -210,14 +213,18 @@ class LayerTW:
             X = X.t().contiguous()
         self.x_layout = x_layout
         self.X = [X] + [X.clone() for _ in range(copies - 1)]
-        self.Y = [torch.empty((d["M"], d["N"]), dtype=torch.float16, device=dev) for _ in range(copies)]
+        yshape = (d["N"], d["M"]) if y_nm else (d["M"], d["N"])
+        self.Y = [torch.empty(yshape, dtype=torch.float16, device=dev) for _ in range(copies)]
         ws = spg.tw_workspace_size(d["M"], d["K"], x_layout)
         self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
 
     def run(self, i, X=None, Y=None):
         X = self.X[i] if X is None else X
         Y = self.Y[i] if Y is None else Y
-        self.spg.spgemm_tw_f16(X, self.desc, self.x_layout, Y=Y, workspace=self.ws, M=self.d["M"])
+        if self.y_nm:
+            self.spg.spgemm_tw_f16_yt(X, self.desc, self.x_layout, Yt=Y, workspace=self.ws, M=self.d["M"])
+        else:
+            self.spg.spgemm_tw_f16(X, self.desc, self.x_layout, Y=Y, workspace=self.ws, M=self.d["M"])
 
 
 def tw_algorithmic(layers_tw):
@@ -249,10 +256,12 @@ def run_ours(args, rank, world, local_rank):
         step_bytes = sum(algorithmic_bytes(d, kind) for d in inputs)
     copies = max(args.copies, int(math.ceil(3 * L2_BYTES / step_bytes)))
     if kind == "tw_f16":
-        layers = [LayerTW(spg, d, copies, spg.SPG_X_KM if args.x_km else spg.SPG_X_MK) for d in inputs]
+        layers = [LayerTW(spg, d, copies, spg.SPG_X_KM if args.x_km else spg.SPG_X_MK, args.y_nm) for d in inputs]
         flops_alg, bytes_alg = tw_algorithmic(layers)
     else:
-        layers = [Layer24(spg, d, kind, copies) for d in inputs]
+        if args.y_nm and kind not in ("24_f16", "24_bf16"):
+            raise SystemExit("--y-nm applies to the 16-bit 2:4 and tile-wise workloads")
+        layers = [Layer24(spg, d, kind, copies, args.y_nm) for d in inputs]
         flops_alg = layer_flops(inputs) / 2.0
         bytes_alg = sum(algorithmic_bytes(d, kind) for d in inputs)
     flops_dense = layer_flops(inputs)
@@ -368,6 +377,7 @@ def run_ours(args, rank, world, local_rank):
                    "l2": f"inputs larger than L2: {copies} rotating buffer sets (X, W, Y) of "
                          f"{step_bytes / 1e6:.1f} MB per step, {copies * step_bytes / 1e6:.0f} MB in all",
                    "launch": "timed steps replayed from CUDA graphs of the library launches",
+                   "layouts": f"X {'[K, M]' if args.x_km else '[M, K]'}, Y {'[N, M] (transposed)' if args.y_nm else '[M, N]'}",
                    "parallelism": f"dp{world} (each rank its own batch, no collective)"},
         "effective_tflops": world * flops_alg * args.steps / (total_ms * 1e-3) / 1e12,
         "per_layer_us": [1e3 * v for v in lay_ms],
@@ -491,6 +501,8 @@ def main():
     ap.add_argument("--workload", default="vitb_mlp_f16", choices=sorted(gen.CONFIGS))
     ap.add_argument("--copies", type=int, default=3)
     ap.add_argument("--x-km", action="store_true", help="tile-wise: activations already [K, M]")
+    ap.add_argument("--y-nm", action="store_true",
+                    help="write Y^T [N, M] (the transpose a following tile-wise layer reads, fused into the GEMM)")
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

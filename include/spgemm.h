@@ -122,6 +122,20 @@ spg_status spgemm_24_f16(const void* X, int64_t ldx, const void* Wv, const uint8
                          spg_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * spgemm_24_f16_yt  [GPUSQ, Abstract; TW, slide "Transpose": the transpose
+ * the next tile-wise layer needs, fused into the producing layer]
+ *
+ * spgemm_24_f16 writing the transpose of Y: Yt[n][m] = Y[m][n], Yt [N, M]
+ * with pitch ldyt >= M.  A tile-wise layer that follows reads Yt directly as
+ * its [K, M] activations (spgemm_tw_f16 with SPG_X_KM), with no transpose.
+ * Same arithmetic, bit-identical values.  Same limits as spgemm_24_f16 with
+ * Y replaced by Yt: Yt 16-byte aligned, ldyt in bytes a multiple of 16.
+ * ------------------------------------------------------------------------- */
+spg_status spgemm_24_f16_yt(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,
+                            void* Yt, int64_t ldyt, int64_t M, int64_t N, int64_t K, spg_dtype dtype,
+                            spg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * spgemm_24_s8  [GPUSQ, Abstract: "2:4 sparse calculation with integer tensors"]
  *
  * acc[m][n] = sum_k X[m][k] * Wm[n][k] in exact int32 on the 2:4 sparse
@@ -225,6 +239,15 @@ size_t tw_workspace_size(int64_t M, int64_t K, int x_layout);
  * ldy >= N; ws_bytes >= tw_workspace_size(M, K, x_layout). */
 spg_status spgemm_tw_f16(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Y,
                          int64_t ldy, int64_t M, void* workspace, size_t ws_bytes, spg_stream_t stream);
+
+/* Tile-wise GEMM writing the transpose of Y [TW, slide "Transpose": with
+ * the transposes fused, a chain of tile-wise layers never leaves the [K, M]
+ * activation layout].  Yt[n][m] = Y[m][n] with Y as spgemm_tw_f16 computes
+ * it (bit-identical values, pruned columns of Y = rows of Yt written as +0).
+ * Yt fp16 [N, M], pitch ldyt >= M, 16-byte aligned, ldyt a multiple of 8.
+ * Other arguments and limits as spgemm_tw_f16. */
+spg_status spgemm_tw_f16_yt(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Yt,
+                            int64_t ldyt, int64_t M, void* workspace, size_t ws_bytes, spg_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * spgemm_tw_f16_noalloc  (no counterpart on the pages: an interface addition)

@@ -47,6 +47,7 @@ SIGNATURES = {
     "sparse_prune_24": (ctypes.c_int, [_p, _i64, _p, _i64, _i64, _i64, ctypes.c_int, _p]),
     "sparse_compress_24": (ctypes.c_int, [_p, _i64, _p, _p, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_f16": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
+    "spgemm_24_f16_yt": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_s8": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _p, _i64, ctypes.c_int, _i64, _i64, _i64, _p]),
     "tw_query_sizes": (ctypes.c_int, [_i64, _i64, _i32, _i64, ctypes.POINTER(_i32), ctypes.POINTER(SpgTwSizes)]),
     "tw_reorganize": (ctypes.c_int, [_p, _i64, _i64, ctypes.POINTER(_i32), ctypes.POINTER(SpgTwDesc), _p, _sz,
@@ -54,6 +55,8 @@ SIGNATURES = {
     "tw_workspace_size": (_sz, [_i64, _i64, ctypes.c_int]),
     "spgemm_tw_f16": (ctypes.c_int, [_p, _i64, ctypes.c_int, ctypes.POINTER(SpgTwDesc), _p, _i64, _i64, _p,
                                      _sz, _p]),
+    "spgemm_tw_f16_yt": (ctypes.c_int, [_p, _i64, ctypes.c_int, ctypes.POINTER(SpgTwDesc), _p, _i64, _i64, _p,
+                                        _sz, _p]),
     "spgemm_tw_f16_noalloc": (ctypes.c_int, [_p, _i64, ctypes.POINTER(SpgTwDesc), _p, _i64, _i64, _p]),
 }
 
@@ -152,6 +155,19 @@ def spgemm_24_f16(X, Wv, meta, bias=None, Y=None, stream=None):
     return Y
 
 
+def spgemm_24_f16_yt(X, Wv, meta, bias=None, Yt=None, stream=None):
+    """Yt [N, M] = (X [M, K] . decompress(Wv, meta)^T (+ bias))^T, fp16 or bf16."""
+    import torch
+    M, K = X.shape
+    N = Wv.shape[0]
+    if Yt is None:
+        Yt = torch.empty((N, M), dtype=X.dtype, device=X.device)
+    _check("spgemm_24_f16_yt", lib().spgemm_24_f16_yt(
+        _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(bias), _ptr(Yt), Yt.stride(0), M, N, K,
+        _dtype_code(X), _stream(stream)))
+    return Yt
+
+
 def spgemm_24_s8(X, Wv, meta, scale=None, bias=None, Y=None, out_mode=SPG_OUT_F16, stream=None):
     """int8 2:4 GEMM; out_mode SPG_OUT_F16 (dequantised fp16) or SPG_OUT_S32 (raw int32)."""
     import torch
@@ -221,6 +237,24 @@ def spgemm_tw_f16(X, desc: TwDesc, x_layout=SPG_X_MK, Y=None, workspace=None, M:
         _ptr(X), X.stride(0), x_layout, ctypes.byref(desc.c), _ptr(Y), Y.stride(0), M, _ptr(workspace),
         ws if workspace is not None else 0, _stream(stream)))
     return Y
+
+
+def spgemm_tw_f16_yt(X, desc: TwDesc, x_layout=SPG_X_MK, Yt=None, workspace=None, M: Optional[int] = None,
+                     stream=None):
+    """Tile-wise GEMM writing Yt [N, M] = Y^T (the [K, M] activations of a following tile-wise layer)."""
+    import torch
+    if M is None:
+        M = X.shape[0] if x_layout == SPG_X_MK else X.shape[1]
+    N = desc.sizes.N
+    if Yt is None:
+        Yt = torch.empty((N, M), dtype=torch.float16, device=X.device)
+    ws = tw_workspace_size(M, desc.sizes.K, x_layout)
+    if workspace is None and ws:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=X.device)
+    _check("spgemm_tw_f16_yt", lib().spgemm_tw_f16_yt(
+        _ptr(X), X.stride(0), x_layout, ctypes.byref(desc.c), _ptr(Yt), Yt.stride(0), M, _ptr(workspace),
+        ws if workspace is not None else 0, _stream(stream)))
+    return Yt
 
 
 def spgemm_tw_f16_noalloc(X, desc: TwDesc, Y=None, stream=None):

@@ -64,6 +64,11 @@ uint32_t* device_error_word() {
 
 bool make_tmap_2d(CUtensorMap* map, const void* base, int esize, uint64_t cols, uint64_t rows,
                   uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
+  return make_tmap_2d_swz(map, base, esize, cols, rows, pitch_bytes, box_cols, box_rows, swizzle128 ? 128 : 0);
+}
+
+bool make_tmap_2d_swz(CUtensorMap* map, const void* base, int esize, uint64_t cols, uint64_t rows,
+                      uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes) {
   std::call_once(g_encode_once, load_encode);
   if (!g_encode) return false;
   CUtensorMapDataType dt = esize == 1   ? CU_TENSOR_MAP_DATA_TYPE_UINT8
@@ -75,7 +80,10 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, int esize, uint64_t cols, 
   cuuint32_t estr[2] = {1, 1};
   CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
                         CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                        swizzle_bytes == 128  ? CU_TENSOR_MAP_SWIZZLE_128B
+                        : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                        : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                              : CU_TENSOR_MAP_SWIZZLE_NONE,
                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }

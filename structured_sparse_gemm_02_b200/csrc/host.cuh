@@ -24,6 +24,10 @@ uint32_t* device_error_word();
 bool make_tmap_2d(CUtensorMap* map, const void* base, int esize, uint64_t cols, uint64_t rows,
                   uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows, bool swizzle128);
 
+// As make_tmap_2d with the shared-memory swizzle given in bytes (0, 32, 64 or 128).
+bool make_tmap_2d_swz(CUtensorMap* map, const void* base, int esize, uint64_t cols, uint64_t rows,
+                      uint64_t pitch_bytes, uint32_t box_cols, uint32_t box_rows, int swizzle_bytes);
+
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 inline spg_status launch_status() {

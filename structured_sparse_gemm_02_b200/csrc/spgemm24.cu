@@ -35,7 +35,10 @@
 namespace spg {
 namespace gemm24 {
 
-enum OutKind { OUT_F16 = 0, OUT_BF16 = 1, OUT_S32 = 2 };
+// Output kinds: Y [M][N] in fp16 / bf16 / int32, or the transpose Y^T [N][M]
+// in fp16 / bf16 (the layout a following tile-wise layer reads as its
+// activations, so that layer needs no transpose).
+enum OutKind { OUT_F16 = 0, OUT_BF16 = 1, OUT_S32 = 2, OUT_F16_T = 3, OUT_BF16_T = 4 };
 
 // Pair tile: 256 weight rows (128 per CTA of the cluster pair) x BN rows of X
 // (BN/2 loaded by each CTA).  STAGES is the deepest operand ring that fits.
@@ -50,6 +53,8 @@ struct Cfg {
   static constexpr int MCP_BYTES = kInt8 ? 0 : 2048;      // fp16/bf16: metadata in tcgen05.cp order
   static constexpr int MCOLS = kInt8 ? 8 : 4;          // TMEM columns of metadata per stage
   static constexpr int OUT_ES = OUT == OUT_S32 ? 4 : 2;
+  static constexpr bool YT = OUT == OUT_F16_T || OUT == OUT_BF16_T;  // Y^T: stored from registers
+  static constexpr bool OUT_BF = OUT == OUT_BF16 || OUT == OUT_BF16_T;
   // staging per epilogue warp: 16-bit outputs double-buffer a 4 KB box per warp
   // pair (2 KB per warp and buffer); int32 outputs one 4 KB box per warp
   static constexpr int EPI_BUF = OUT_ES == 2 ? 2 * 2048 : 4096;
@@ -142,7 +147,7 @@ __device__ __forceinline__ uint32_t convert_out(uint32_t acc, float badd, float 
     float v = __fmul_rn(__int2float_rn(static_cast<int>(acc)), sc);
     if (has_bias) v = __fadd_rn(v, badd);
     return __half_as_ushort(__float2half_rn(v));
-  } else if constexpr (OUT == OUT_BF16) {
+  } else if constexpr (OUT == OUT_BF16 || OUT == OUT_BF16_T) {
     return __bfloat16_as_ushort(__float2bfloat16_rn(__fadd_rn(__uint_as_float(acc), badd)));
   } else {
     return __half_as_ushort(__float2half_rn(__fadd_rn(__uint_as_float(acc), badd)));
@@ -167,7 +172,7 @@ __device__ __forceinline__ uint32_t convert_pair16(uint32_t a0, uint32_t a1, flo
     v1 = __fadd_rn(__uint_as_float(a1), badd);
   }
   uint32_t w;
-  if constexpr (OUT == OUT_BF16)
+  if constexpr (OUT == OUT_BF16 || OUT == OUT_BF16_T)
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(v1), "f"(v0));
   else
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(v1), "f"(v0));
@@ -410,6 +415,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     const bool pair_lead = (q & 1) == 0;
     bool staged = false;  // int32: a TMA store from buf may still be reading it
     uint32_t nst = 0;     // 16-bit: pair boxes stored so far
+    uint32_t nyt = 0;     // Y^T: boxes this warp stored so far
     int i = 0;
     for (int t = pair; t < total; t += npairs, ++i) {
       const int n0 = (t % NT) * 256 + 128 * int(rank), m0 = (t / NT) * BN;
@@ -459,6 +465,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           // packed pairs (rows 2j, 2j+1) kept in h[0..15]
 #pragma unroll
           for (int j = 0; j < 16; ++j) h[j] = convert_pair16<OUT, kInt8>(h[2 * j], h[2 * j + 1], badd, sc, has_bias);
+        }
+        if constexpr (C::YT) {
+          // Y^T [N][M]: lane n holds rows mb..mb+31 of output column n, i.e.
+          // 64 contiguous bytes of row n of Y^T.  The warp's [32 n][32 m]
+          // block goes to a double-buffered 2 KB box (64-byte swizzle: 16-byte
+          // chunk k of row r at chunk k ^ ((r >> 1) & 3)) and out by one TMA
+          // store, which clips rows >= N.  A chunk that crosses M (the
+          // inner dimension, where the store would not stop at the exact
+          // element) is written by element stores instead.
+          if (mb + 32 > M) {
+            if (n < N) {
+              uint16_t* dst = static_cast<uint16_t*>(Yp) + int64_t(n) * ldy + mb;
+#pragma unroll
+              for (int k = 0; k < 32; ++k)
+                if (mb + k < M) dst[k] = static_cast<uint16_t>((k & 1) ? (h[k >> 1] >> 16) : (h[k >> 1] & 0xFFFFu));
+            }
+            continue;
+          }
+          const uint32_t box = smem_addr(buf) + (nyt & 1) * 2048u;
+          if (nyt >= 2) {
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t a = box + uint32_t(lane) * 64u + (uint32_t(k ^ ((lane >> 1) & 3)) << 4);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(h[4 * k]), "r"(h[4 * k + 1]),
+                         "r"(h[4 * k + 2]), "r"(h[4 * k + 3])
+                         : "memory");
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d_saddr(&tmY, box, mb, nb);
+            bulk_commit();
+          }
+          __syncwarp();
+          ++nyt;
+          continue;
         }
         if (C::OUT_ES == 4 && full_n) {
           // int32: one [32][32] box (128 B rows) per warp
@@ -568,8 +613,9 @@ spg_status launch(const void* X, int64_t ldx, const void* Wv, const uint8_t* met
   if (!make_tmap_2d(&tmA, Wv, es, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2) * es, 128 / es, 128, true) ||
       !make_tmap_2d(&tmB, X, es, uint64_t(K), uint64_t(M), uint64_t(ldx) * es, 128 / es, C::BNH, true) ||
       !make_tmap_2d(&tmE, meta, 1, uint64_t(K / 8), uint64_t(N), uint64_t(K / 8), 16, 128, false) ||
-      !make_tmap_2d(&tmY, Y, C::OUT_ES, uint64_t(N), uint64_t(M), uint64_t(ldy) * C::OUT_ES,
-                    C::OUT_ES == 2 ? 64 : 32, 32, C::OUT_ES == 2))
+      !(C::YT ? make_tmap_2d_swz(&tmY, Y, 2, uint64_t(M), uint64_t(N), uint64_t(ldy) * 2, 32, 32, 64)
+              : make_tmap_2d(&tmY, Y, C::OUT_ES, uint64_t(N), uint64_t(M), uint64_t(ldy) * C::OUT_ES,
+                             C::OUT_ES == 2 ? 64 : 32, 32, C::OUT_ES == 2)))
     return SPG_ERR_CUDA;
   uint32_t* err = device_error_word();
   if (!err) return SPG_ERR_CUDA;
@@ -596,9 +642,9 @@ spg_status dispatch(const void* X, int64_t ldx, const void* Wv, const uint8_t* m
 }
 
 spg_status validate_common(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, void* Y, int64_t ldy,
-                           int64_t M, int64_t N, int64_t K, int es, int out_es, int kstep) {
+                           int64_t M, int64_t N, int64_t K, int es, int out_es, int kstep, bool y_transposed = false) {
   if (!X || !Wv || !meta || !Y) return SPG_ERR_INVALID_ARG;
-  if (M <= 0 || N <= 0 || K <= 0 || ldx < K || ldy < N) return SPG_ERR_INVALID_ARG;
+  if (M <= 0 || N <= 0 || K <= 0 || ldx < K || ldy < (y_transposed ? M : N)) return SPG_ERR_INVALID_ARG;
   if (K % kstep || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
     return SPG_ERR_UNSUPPORTED_SHAPE;
   if ((N + 127) / 128 * ((M + 31) / 32) >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
@@ -626,6 +672,23 @@ spg_status spgemm_24_f16(const void* X, int64_t ldx, const void* Wv, const uint8
   auto s = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == SPG_F16) return dispatch<false, false, OUT_F16>(X, ldx, Wv, meta, bias, nullptr, Y, ldy, M, N, K, s);
   return dispatch<false, true, OUT_BF16>(X, ldx, Wv, meta, bias, nullptr, Y, ldy, M, N, K, s);
+}
+
+spg_status spgemm_24_f16_yt(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,
+                            void* Yt, int64_t ldyt, int64_t M, int64_t N, int64_t K, spg_dtype dtype,
+                            spg_stream_t stream) {
+  using namespace spg;
+  using namespace spg::gemm24;
+  if (dtype != SPG_F16 && dtype != SPG_BF16) return SPG_ERR_INVALID_ARG;
+  spg_status st = validate_common(X, ldx, Wv, meta, Yt, ldyt, M, N, K, 2, 2, 128, true);
+  if (st != SPG_OK) return st;
+  if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;
+  st = check_device();
+  if (st != SPG_OK) return st;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == SPG_F16)
+    return dispatch<false, false, OUT_F16_T>(X, ldx, Wv, meta, bias, nullptr, Yt, ldyt, M, N, K, s);
+  return dispatch<false, true, OUT_BF16_T>(X, ldx, Wv, meta, bias, nullptr, Yt, ldyt, M, N, K, s);
 }
 
 spg_status spgemm_24_s8(const int8_t* X, int64_t ldx, const int8_t* Wv, const uint8_t* meta, const float* scale,

@@ -275,7 +275,7 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 __global__ void __launch_bounds__(THREADS, 1)
     tw_gemm_kernel(const __grid_constant__ CUtensorMap tmWc, const __grid_constant__ CUtensorMap tmY64,
                    const __grid_constant__ CUtensorMap tmY8, const uint16_t* __restrict__ xt, int64_t ldt,
-                   uint16_t* __restrict__ Y, int64_t ldy, int vec_ok, int M, int Nk, int T,
+                   uint16_t* __restrict__ Y, int64_t ldy, int vec_ok, int y_nm, int M, int Nk, int T,
                    const int* __restrict__ offsetn,
                    const int* __restrict__ tile_n0, const int* __restrict__ tile_kofs,
                    const int* __restrict__ offsetk, uint32_t* err) {
@@ -485,6 +485,42 @@ __global__ void __launch_bounds__(THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[b]);
 
+      if (y_nm) {
+        // Y^T [N][M]: this lane's kept column nj is row nj of Y^T, and its 64
+        // rows m are 128 contiguous bytes of that row, stored from registers;
+        // the pruned columns it owns (its gap, and the tile's lead for j = 0)
+        // are rows of zeros.  rows is a multiple of 8 (M % 8 == 0).
+        if (valid && rows > 0) {
+          uint16_t* yrow = Y + int64_t(nj) * ldy + mb;
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            uint32_t w[16];
+#pragma unroll
+            for (int p = 0; p < 16; ++p) {
+              const float v0 = __uint_as_float(r[cc][2 * p]), v1 = __uint_as_float(r[cc][2 * p + 1]);
+              asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w[p]) : "f"(v1), "f"(v0));
+            }
+            if (32 * cc + 32 <= rows) {
+              uint4* d4 = reinterpret_cast<uint4*>(yrow + 32 * cc);
+#pragma unroll
+              for (int p = 0; p < 4; ++p) d4[p] = make_uint4(w[4 * p], w[4 * p + 1], w[4 * p + 2], w[4 * p + 3]);
+            } else if (32 * cc < rows) {
+              uint4* d4 = reinterpret_cast<uint4*>(yrow + 32 * cc);
+              for (int p = 0; p < (rows - 32 * cc) / 8; ++p) d4[p] = make_uint4(w[4 * p], w[4 * p + 1], w[4 * p + 2], w[4 * p + 3]);
+            }
+          }
+          const int gap_end = j + 1 < Gt ? offsetn[j0 + j + 1] : n1;
+          auto zero_row = [&](int z) {
+            uint4* d4 = reinterpret_cast<uint4*>(Y + int64_t(z) * ldy + mb);
+            for (int e = 0; e < rows / 8; ++e) d4[e] = make_uint4(0u, 0u, 0u, 0u);
+          };
+          for (int z = nj + 1; z < gap_end; ++z) zero_row(z);
+          if (j == 0)
+            for (int z = n0; z < nj; ++z) zero_row(z);
+        }
+        continue;
+      }
+
       // Windows: zero, place kept columns, store.  Layout of a window of ww
       // columns (a multiple of 8): nw blocks [64 rows][64 columns] then nn
       // blocks [64 rows][8 columns], the shapes of the two TMA store boxes.
@@ -625,12 +661,12 @@ spg_status query(int64_t N, int64_t K, int32_t G, int64_t n_pruned, const int32_
 // Tensor maps and launch of the run-time GEMM over transposed activations
 // xt [K][ldt] (shared by the entry points below).
 spg_status launch_gemm(const uint16_t* xt, int64_t ldt, const spg_tw_desc* desc, uint16_t* Y, int64_t ldy,
-                       int64_t M, cudaStream_t s) {
+                       int64_t M, cudaStream_t s, bool y_nm = false) {
   CUtensorMap tmWc, tmY64, tmY8;
   const uint64_t wc_rows = uint64_t(desc->offsetk_len / kKBlock) * kG;
   if (!make_tmap_2d(&tmWc, desc->Wc, 2, kKBlock, wc_rows, kKBlock * 2, kKBlock, kG, true)) return SPG_ERR_CUDA;
   // Y leaves through TMA when its rows are 16-byte aligned; otherwise by element stores only
-  const int vec_ok = aligned(Y, 16) && (ldy % 8) == 0;
+  const int vec_ok = !y_nm && aligned(Y, 16) && (ldy % 8) == 0;
   if (vec_ok) {
     if (!make_tmap_2d(&tmY64, Y, 2, uint64_t(desc->N), uint64_t(M), uint64_t(ldy) * 2, 64, RG, false) ||
         !make_tmap_2d(&tmY8, Y, 2, uint64_t(desc->N), uint64_t(M), uint64_t(ldy) * 2, 8, RG, false))
@@ -644,9 +680,43 @@ spg_status launch_gemm(const uint16_t* xt, int64_t ldt, const spg_tw_desc* desc,
   if (!smem_attr_set()) return SPG_ERR_CUDA;
   const int64_t units = int64_t(desc->T) * ((M + BN - 1) / BN);
   const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
-  tw_gemm_kernel<<<grid, THREADS, SMEM, s>>>(tmWc, tmY64, tmY8, xt, ldt, Y, ldy, vec_ok, int(M), int(desc->Nk), desc->T,
+  tw_gemm_kernel<<<grid, THREADS, SMEM, s>>>(tmWc, tmY64, tmY8, xt, ldt, Y, ldy, vec_ok, y_nm ? 1 : 0, int(M),
+                                              int(desc->Nk), desc->T,
                                          desc->offsetn, desc->tile_n0, desc->tile_kofs, desc->offsetk, err);
   return launch_status();
+}
+
+// Validation, the optional explicit transpose and the GEMM launch shared by
+// spgemm_tw_f16 (Y [M][N], y_nm false) and spgemm_tw_f16_yt (Y^T [N][M]).
+spg_status run(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Y, int64_t ldy, int64_t M,
+               void* workspace, size_t ws_bytes, spg_stream_t stream, bool y_nm) {
+  if (!X || !desc || !Y) return SPG_ERR_INVALID_ARG;
+  if (x_layout != SPG_X_MK && x_layout != SPG_X_KM) return SPG_ERR_INVALID_ARG;
+  const int64_t N = desc->N, K = desc->K;
+  if (M <= 0 || N <= 0 || K <= 0 || ldy < (y_nm ? M : N)) return SPG_ERR_INVALID_ARG;
+  if (desc->G != kG || desc->T <= 0 || desc->offsetk_len <= 0 || desc->offsetk_len % kKBlock) return SPG_ERR_INVALID_ARG;
+  if (!desc->offsetn || !desc->tile_n0 || !desc->tile_kofs || !desc->offsetk || !desc->Wc) return SPG_ERR_INVALID_ARG;
+  if (x_layout == SPG_X_MK ? ldx < K : ldx < M) return SPG_ERR_INVALID_ARG;
+  if (M % 8 || M >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned(X, 16) || !aligned(Y, 2) || ldx % 8) return SPG_ERR_MISALIGNED;
+  if (y_nm && (!aligned(Y, 16) || ldy % 8)) return SPG_ERR_MISALIGNED;
+  if (x_layout == SPG_X_MK) {
+    if (!workspace || ws_bytes < tw_workspace_size(M, K, x_layout)) return SPG_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return SPG_ERR_MISALIGNED;
+  }
+  spg_status st = check_device();
+  if (st != SPG_OK) return st;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  const uint16_t* xt = static_cast<const uint16_t*>(X);
+  int64_t ldt = ldx;
+  if (x_layout == SPG_X_MK) {
+    uint16_t* ws = static_cast<uint16_t*>(workspace);
+    dim3 grid(static_cast<unsigned>((K + 63) / 64), static_cast<unsigned>((M + 63) / 64));
+    transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(static_cast<const uint16_t*>(X), ldx, int(M), int(K), ws, M);
+    xt = ws;
+    ldt = M;
+  }
+  return launch_gemm(xt, ldt, desc, static_cast<uint16_t*>(Y), ldy, M, s, y_nm);
 }
 
 // ---- scratch for the entry point that allocates nothing ------------------------------------
@@ -740,34 +810,13 @@ spg_status tw_reorganize(const void* W, int64_t ldw, int64_t n_pruned, const int
 
 spg_status spgemm_tw_f16(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Y, int64_t ldy,
                          int64_t M, void* workspace, size_t ws_bytes, spg_stream_t stream) {
-  using namespace spg;
-  using namespace spg::tw;
-  if (!X || !desc || !Y) return SPG_ERR_INVALID_ARG;
-  if (x_layout != SPG_X_MK && x_layout != SPG_X_KM) return SPG_ERR_INVALID_ARG;
-  const int64_t N = desc->N, K = desc->K;
-  if (M <= 0 || N <= 0 || K <= 0 || ldy < N) return SPG_ERR_INVALID_ARG;
-  if (desc->G != kG || desc->T <= 0 || desc->offsetk_len <= 0 || desc->offsetk_len % kKBlock) return SPG_ERR_INVALID_ARG;
-  if (!desc->offsetn || !desc->tile_n0 || !desc->tile_kofs || !desc->offsetk || !desc->Wc) return SPG_ERR_INVALID_ARG;
-  if (x_layout == SPG_X_MK ? ldx < K : ldx < M) return SPG_ERR_INVALID_ARG;
-  if (M % 8 || M >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
-  if (!aligned(X, 16) || !aligned(Y, 2) || ldx % 8) return SPG_ERR_MISALIGNED;
-  if (x_layout == SPG_X_MK) {
-    if (!workspace || ws_bytes < tw_workspace_size(M, K, x_layout)) return SPG_ERR_INVALID_ARG;
-    if (!aligned(workspace, 16)) return SPG_ERR_MISALIGNED;
-  }
-  spg_status st = check_device();
-  if (st != SPG_OK) return st;
-  auto s = reinterpret_cast<cudaStream_t>(stream);
-  const uint16_t* xt = static_cast<const uint16_t*>(X);
-  int64_t ldt = ldx;
-  if (x_layout == SPG_X_MK) {
-    uint16_t* ws = static_cast<uint16_t*>(workspace);
-    dim3 grid(static_cast<unsigned>((K + 63) / 64), static_cast<unsigned>((M + 63) / 64));
-    transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(static_cast<const uint16_t*>(X), ldx, int(M), int(K), ws, M);
-    xt = ws;
-    ldt = M;
-  }
-  return launch_gemm(xt, ldt, desc, static_cast<uint16_t*>(Y), ldy, M, s);
+  return spg::tw::run(X, ldx, x_layout, desc, Y, ldy, M, workspace, ws_bytes, stream, false);
+}
+
+// Y^T [N][M] output: the transpose a following tile-wise layer needs is fused here.
+spg_status spgemm_tw_f16_yt(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Yt,
+                            int64_t ldyt, int64_t M, void* workspace, size_t ws_bytes, spg_stream_t stream) {
+  return spg::tw::run(X, ldx, x_layout, desc, Yt, ldyt, M, workspace, ws_bytes, stream, true);
 }
 
 // Tile-wise GEMM on [M, K] activations for callers that cannot allocate

@@ -67,3 +67,13 @@ def test_validation_rejects_before_touching_the_device():
     assert L.sparse_prune_24(16, 6, 16, 6, 2, 6, 0, None) == 2                               # K % 4
     assert L.sparse_compress_24(16, 12, 16, 16, 2, 12, 0, None) == 2                         # K % 8
     assert L.sparse_prune_24(16, 8, 16, 8, 0, 8, 0, None) == 0                               # empty: no-op
+    # transposed outputs: the pitch of Y^T covers M, not N
+    assert L.spgemm_24_f16_yt(16, 256, 16, 16, None, 16, 32, 64, 256, 256, 0, None) == 1  # ldyt < M
+    assert L.spgemm_24_f16_yt(16, 256, 16, 16, None, 16, 68, 68, 256, 256, 0, None) == 3  # ldyt*2 % 16
+    desc = spg.SpgTwDesc()
+    desc.N, desc.K, desc.Nk, desc.G, desc.T, desc.offsetk_len = 768, 768, 691, 128, 6, 1536
+    for f in ("offsetn", "tile_n0", "tile_kofs", "k_per_tile", "offsetk", "Wc"):
+        setattr(desc, f, 256)
+    assert L.spgemm_tw_f16_yt(16, 64, 1, ctypes.byref(desc), 16, 32, 64, None, 0, None) == 1  # ldyt < M
+    assert L.spgemm_tw_f16_yt(16, 64, 1, ctypes.byref(desc), 18, 64, 64, None, 0, None) == 3  # Yt not 16-B aligned
+    assert L.spgemm_tw_f16_yt(16, 64, 1, ctypes.byref(desc), 16, 68, 64, None, 0, None) == 3  # ldyt % 8
