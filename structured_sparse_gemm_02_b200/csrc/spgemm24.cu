@@ -13,8 +13,9 @@
 //              every stage into a STAGES-deep ring that runs across tiles
 //   warp 1     fp16/bf16 only: rearranges each stage's metadata into the
 //              order the tensor cores read it (permute_meta_f16)
-//   warp 2     TMEM owner and MMA issuer: tcgen05.cp (metadata into tensor
-//              memory), tcgen05.mma.sp into one of two accumulators
+//   warp 2     TMEM owner and MMA issuer (one thread of the leader CTA):
+//              tcgen05.cp (metadata into tensor memory), tcgen05.mma.sp into
+//              one of two accumulators
 //   warp 3     idle
 //   warps 4-7  epilogue: tcgen05.ld of a finished accumulator (released as
 //              soon as it is read), bias / dequant, convert, TMA store of
@@ -338,7 +339,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     }
   } else if (warp == 2) {
     // ---------------- MMA issuer (leader CTA) ----------------
-    if (leader) {
+    // One thread runs the whole loop: the waits are single-thread bounded
+    // waits, because a warp-wide wait and vote between two groups of MMAs
+    // costs more than its share of the tensor pipe's time.
+    if (leader && lane == 0) {
       constexpr uint32_t kFmt = kInt8 ? 1u : (kBF16 ? 1u : 0u);
       constexpr uint32_t kCFmt = kInt8 ? 2u : 1u;
       uint32_t g = 0;
@@ -346,56 +350,51 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       bool ok = true;
       for (int t = pair; ok && t < total; t += npairs, ++i) {
         const int b = i & 1;
-        if (i >= 2 && !mbar_wait_warp(&acc_empty[b], ((i >> 1) - 1) & 1, abort_flag, err, ERR_WAIT_ACC_FREE)) break;
+        if (i >= 2 && !mbar_wait(&acc_empty[b], ((i >> 1) - 1) & 1, abort_flag, err, ERR_WAIT_ACC_FREE)) break;
         tc_fence_after();
         const uint32_t acc = tmem + uint32_t(b * BN);
         for (int kb = 0; kb < KB; ++kb, ++g) {
           const int s = g % STAGES;
           const uint32_t ph = (g / STAGES) & 1;
-          if (!mbar_wait_warp(&full[s], ph, abort_flag, err, ERR_WAIT_FULL)) {
+          if (!mbar_wait(&full[s], ph, abort_flag, err, ERR_WAIT_FULL)) {
             ok = false;
             break;
           }
           if constexpr (!kInt8) {
-            if (!mbar_wait_warp(&meta_full[s], ph, abort_flag, err, ERR_WAIT_META)) {
+            if (!mbar_wait(&meta_full[s], ph, abort_flag, err, ERR_WAIT_META)) {
               ok = false;
               break;
             }
           }
           tc_fence_after();
-          if (lane == 0) {
-            const uint32_t a_s = smem_addr(smem + C::OFF_A + s * C::A_BYTES);
-            const uint32_t b_s = smem_addr(smem + C::OFF_B + s * C::B_BYTES);
-            const uint32_t ecol = tmem + C::META_COL + (g & 1) * C::MCOLS;
-            if constexpr (kInt8) {
-              const uint32_t e_s = smem_addr(smem + C::OFF_MSTG + s * C::MSTG_BYTES);
-              tc_cp_128x128b_pair(ecol, smem_desc(e_s, 2048, 128, LAYOUT_NONE));
-              tc_cp_128x128b_pair(ecol + 4, smem_desc(e_s + 2048, 2048, 128, LAYOUT_NONE));
-            } else {
-              const uint32_t e_s = smem_addr(smem + C::OFF_MCP + s * C::MCP_BYTES);
-              tc_cp_128x128b_pair(ecol, smem_desc(e_s, 2048, 128, LAYOUT_NONE));
-            }
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint64_t adesc = smem_desc(a_s + 32 * j, 16, 1024, LAYOUT_SW128);
-              const uint64_t bdesc =
-                  smem_desc(b_s + (j >> 1) * (BNH * 128) + (j & 1) * 64, 16, 1024, LAYOUT_SW128);
-              const uint32_t e = kInt8 ? ecol + 2 * j : ecol + (j & ~1);
-              const uint32_t sel = kInt8 ? 0u : uint32_t(j & 1);
-              tc_mma_sp_pair<kInt8>(acc, adesc, bdesc, e, instr_desc(kFmt, kCFmt, 256, BN, true, sel),
-                                    (kb | j) != 0 ? 1u : 0u);
-            }
-            tc_commit_pair(&empty[s], 0x3);
+          const uint32_t a_s = smem_addr(smem + C::OFF_A + s * C::A_BYTES);
+          const uint32_t b_s = smem_addr(smem + C::OFF_B + s * C::B_BYTES);
+          const uint32_t ecol = tmem + C::META_COL + (g & 1) * C::MCOLS;
+          if constexpr (kInt8) {
+            const uint32_t e_s = smem_addr(smem + C::OFF_MSTG + s * C::MSTG_BYTES);
+            tc_cp_128x128b_pair(ecol, smem_desc(e_s, 2048, 128, LAYOUT_NONE));
+            tc_cp_128x128b_pair(ecol + 4, smem_desc(e_s + 2048, 2048, 128, LAYOUT_NONE));
+          } else {
+            const uint32_t e_s = smem_addr(smem + C::OFF_MCP + s * C::MCP_BYTES);
+            tc_cp_128x128b_pair(ecol, smem_desc(e_s, 2048, 128, LAYOUT_NONE));
           }
-          __syncwarp();
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t adesc = smem_desc(a_s + 32 * j, 16, 1024, LAYOUT_SW128);
+            const uint64_t bdesc = smem_desc(b_s + (j >> 1) * (BNH * 128) + (j & 1) * 64, 16, 1024, LAYOUT_SW128);
+            const uint32_t e = kInt8 ? ecol + 2 * j : ecol + (j & ~1);
+            const uint32_t sel = kInt8 ? 0u : uint32_t(j & 1);
+            tc_mma_sp_pair<kInt8>(acc, adesc, bdesc, e, instr_desc(kFmt, kCFmt, 256, BN, true, sel),
+                                  (kb | j) != 0 ? 1u : 0u);
+          }
+          tc_commit_pair(&empty[s], 0x3);
         }
         if (!ok) break;
-        if (lane == 0) tc_commit_pair(&acc_full[b], 0x3);
-        __syncwarp();
+        tc_commit_pair(&acc_full[b], 0x3);
       }
-      if (lane == 0) tc_commit_pair(mma_done, 0x3);
-      __syncwarp();
+      tc_commit_pair(mma_done, 0x3);
     }
+    __syncwarp();
     // both CTAs: every MMA reading this CTA's shared memory or writing its
     // tensor memory has completed once the leader's final commit arrives
     if (lane == 0) tail_wait(mma_done, 0, err);

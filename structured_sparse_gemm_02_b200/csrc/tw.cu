@@ -391,27 +391,28 @@ __global__ void __launch_bounds__(THREADS, 1)
     __syncwarp();
   } else if (warp == 2) {
     // ---------------- MMA ----------------
-    // kind::f16 dense, fp16 inputs, fp32 accumulate, A K-major, B MN-major, M=128, N=128
+    // kind::f16 dense, fp16 inputs, fp32 accumulate, A K-major, B MN-major, M=128, N=128.
+    // One thread issues, with single-thread bounded waits.
     constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | (1u << 16) | ((BN >> 3) << 17) | ((128 >> 4) << 24);
-    uint32_t g = 0;
-    int i = 0;
-    bool ok = true;
-    for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++i) {
-      const int t = u / MB;
-      const int KB = (tile_kofs[t + 1] - tile_kofs[t]) / kKBlock;
-      const int b = i & 1;
-      if (i >= 2 && !mbar_wait_warp(&acc_empty[b], ((i >> 1) - 1) & 1, abort_flag, err, ERR_WAIT_ACC_FREE)) break;
-      tc_fence_after();
-      const uint32_t acc = tmem + uint32_t(b * BN);
-      for (int kb = 0; kb < KB; ++kb, ++g) {
-        const int s = g % STAGES;
-        if (!mbar_wait_warp(&full[s], (g / STAGES) & 1, abort_flag, err, ERR_WAIT_FULL)) {
-          ok = false;
-          break;
-        }
+    if (lane == 0) {
+      uint32_t g = 0;
+      int i = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < units; u += gridDim.x, ++i) {
+        const int t = u / MB;
+        const int KB = (tile_kofs[t + 1] - tile_kofs[t]) / kKBlock;
+        const int b = i & 1;
+        if (i >= 2 && !mbar_wait(&acc_empty[b], ((i >> 1) - 1) & 1, abort_flag, err, ERR_WAIT_ACC_FREE)) break;
         tc_fence_after();
-        fence_proxy_async_smem();  // the gathered rows were written by cp.async (generic proxy)
-        if (lane == 0) {
+        const uint32_t acc = tmem + uint32_t(b * BN);
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % STAGES;
+          if (!mbar_wait(&full[s], (g / STAGES) & 1, abort_flag, err, ERR_WAIT_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          fence_proxy_async_smem();  // the gathered rows were written by cp.async (generic proxy)
           const uint32_t a_s = smem_addr(smem + s * (A_BYTES + B_BYTES));
           const uint32_t b_s = a_s + A_BYTES;
 #pragma unroll
@@ -422,13 +423,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           tc_commit(&empty[s]);
         }
-        __syncwarp();
+        if (!ok) break;
+        tc_commit(&acc_full[b]);
       }
-      if (!ok) break;
-      if (lane == 0) tc_commit(&acc_full[b]);
-      __syncwarp();
-    }
-    if (lane == 0) {
       tc_commit(mma_done);
       tail_wait(mma_done, 0, err);
     }
