@@ -67,6 +67,15 @@ const char* spg_status_string(spg_status s);
  * SPG_ERR_CUDA if the synchronisation failed, SPG_OK otherwise. */
 spg_status spg_check_device_error(spg_stream_t stream, uint32_t* bits);
 
+/* Self-test of the failure path every kernel uses (no counterpart on the
+ * pages): launches one thread that waits, with the library's bounded wait
+ * and a limit of limit_ns nanoseconds (0 < limit_ns <= 10 s), on an mbarrier
+ * that nothing ever completes.  The wait gives up, records bit 6 in the
+ * device error word and the kernel returns; nothing faults and the context
+ * stays usable.  A following spg_check_device_error() returns
+ * SPG_ERR_TIMEOUT with that bit (and clears it).  Asynchronous on `stream`. */
+spg_status spg_selftest_bounded_wait(int64_t limit_ns, spg_stream_t stream);
+
 /* ---------------------------------------------------------------------------
  * sparse_prune_24  [GPUSQ, Abstract: "2:4 structured pruning"]
  *

@@ -44,6 +44,7 @@ SIGNATURES = {
     "spg_version": (ctypes.c_int, []),
     "spg_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "spg_check_device_error": (ctypes.c_int, [_p, ctypes.POINTER(ctypes.c_uint32)]),
+    "spg_selftest_bounded_wait": (ctypes.c_int, [_i64, _p]),
     "sparse_prune_24": (ctypes.c_int, [_p, _i64, _p, _i64, _i64, _i64, ctypes.c_int, _p]),
     "sparse_compress_24": (ctypes.c_int, [_p, _i64, _p, _p, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_f16": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
@@ -116,6 +117,12 @@ def check_device_error(stream=None) -> int:
     if st not in (0, 6):
         _check("spg_check_device_error", st)
     return int(bits.value)
+
+
+def selftest_bounded_wait(limit_ns: int = 20_000_000, stream=None) -> None:
+    """Launch the self-test whose bounded wait runs out (see spgemm.h); read the
+    result with check_device_error()."""
+    _check("spg_selftest_bounded_wait", lib().spg_selftest_bounded_wait(int(limit_ns), _stream(stream)))
 
 
 def sparse_prune_24(W, Wm=None, stream=None):

@@ -6,6 +6,7 @@
 #include <mutex>
 
 #include "host.cuh"
+#include "sm100.cuh"
 #include "spgemm.h"
 
 namespace spg {
@@ -88,6 +89,21 @@ bool make_tmap_2d_swz(CUtensorMap* map, const void* base, int esize, uint64_t co
   return r == CUDA_SUCCESS;
 }
 
+// One thread waits, with the library's bounded wait and the given limit, on
+// an mbarrier that nothing ever arrives on: the wait gives up, records
+// ERR_WAIT_SELFTEST in the error word and the kernel returns normally.
+__global__ void selftest_wait_kernel(uint32_t* err, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, err, ERR_WAIT_SELFTEST, limit_ns);
+}
+
 }  // namespace spg
 
 extern "C" {
@@ -117,6 +133,16 @@ spg_status spg_check_device_error(spg_stream_t stream, uint32_t* bits) {
   if (v && cudaMemcpyToSymbol(spg::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SPG_ERR_CUDA;
   if (bits) *bits = v;
   return v ? SPG_ERR_TIMEOUT : SPG_OK;
+}
+
+spg_status spg_selftest_bounded_wait(int64_t limit_ns, spg_stream_t stream) {
+  if (limit_ns <= 0 || limit_ns > 10ll * 1000 * 1000 * 1000) return SPG_ERR_INVALID_ARG;
+  spg_status st = spg::check_device();
+  if (st != SPG_OK) return st;
+  uint32_t* err = spg::device_error_word();
+  if (!err) return SPG_ERR_CUDA;
+  spg::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(err, uint64_t(limit_ns));
+  return spg::launch_status();
 }
 
 }  // extern "C"

@@ -21,6 +21,7 @@ enum : uint32_t {
   ERR_WAIT_ACC_FREE = 1u << 3, // MMA waited for the epilogue to drain TMEM
   ERR_WAIT_TAIL = 1u << 4,     // teardown waited for in-flight copies
   ERR_WAIT_META = 1u << 5,     // MMA waited for staged metadata
+  ERR_WAIT_SELFTEST = 1u << 6, // spg_selftest_bounded_wait: the wait that nothing completes
 };
 
 // A single wait may take at most this long before the kernel gives up.
@@ -74,7 +75,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // false (after setting `code` in *err and the block abort flag) if the wait
 // exceeds kWaitLimitNs or another role of the block has already aborted.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t* err, uint32_t code) {
+                                          uint32_t* err, uint32_t code, uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_addr(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
@@ -82,7 +83,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 31u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         if (err) atomicOr(err, code);
         return false;

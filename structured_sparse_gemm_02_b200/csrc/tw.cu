@@ -182,37 +182,50 @@ __global__ void gather_wc_kernel(const uint16_t* __restrict__ W, int64_t ldw, in
 }
 
 // ---- explicit activation transpose X [M, K] -> Xt [K, M] ------------------------------------
-// 64 x 64 tiles through shared memory; 32-bit (two fp16) accesses on both sides.
-__global__ void transpose_kernel(const uint16_t* __restrict__ X, int64_t ldx, int M, int K,
-                                 uint16_t* __restrict__ Xt, int64_t ldt) {
+// One 64 (m) x 64 (k) tile per 256-thread block, 16-byte accesses on both
+// sides (M % 8 == 0, K % 64 == 0, 16-byte aligned rows).  The tile sits in
+// shared memory as 32-bit pairs (k, k+1) with a row pitch of 33 words, so
+// both the row-wise stores and the column-wise reads are free of bank
+// conflicts.  Reads: thread t takes 8 consecutive k of rows t/8 and t/8 + 32.
+// Writes: thread t takes the k pair 2 (t/8) .. +1 and the 8 m of chunk t % 8,
+// so 8 consecutive threads write 128 contiguous bytes of one output row.
+__global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ X, int64_t ldx, int M, int K,
+                                                        uint16_t* __restrict__ Xt, int64_t ldt) {
   __shared__ uint32_t tile[64][33];  // [m][k pair]
   const int m0 = blockIdx.y * 64, k0 = blockIdx.x * 64;
-  const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+  const int t = threadIdx.x;
+  {
+    const int c = t & 7;
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int m = m0 + ty + 8 * r, k = k0 + 2 * tx;
-    uint32_t v = 0;
-    if (m < M && k + 1 < K) {
-      v = *reinterpret_cast<const uint32_t*>(X + int64_t(m) * ldx + k);
-    } else if (m < M && k < K) {
-      v = X[int64_t(m) * ldx + k];
+    for (int h = 0; h < 2; ++h) {
+      const int r = (t >> 3) + 32 * h;
+      if (m0 + r < M) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + int64_t(m0 + r) * ldx + k0 + 8 * c));
+        tile[r][4 * c + 0] = v.x;
+        tile[r][4 * c + 1] = v.y;
+        tile[r][4 * c + 2] = v.z;
+        tile[r][4 * c + 3] = v.w;
+      }
     }
-    tile[ty + 8 * r][tx] = v;
   }
   __syncthreads();
+  const int kp = t >> 3, j = t & 7;  // k pair (k = 2 kp, 2 kp + 1), m chunk
+  if (m0 + 8 * j >= M) return;
+  uint32_t w[8];
 #pragma unroll
-  for (int r = 0; r < 8; ++r) {
-    const int kl = ty + 8 * r, k = k0 + kl;
-    const int m = m0 + 2 * tx;
-    if (k >= K || m >= M) continue;
-    const int sh = 16 * (kl & 1);
-    const uint32_t lo = (tile[2 * tx][kl >> 1] >> sh) & 0xFFFFu;
-    const uint32_t hi = (tile[2 * tx + 1][kl >> 1] >> sh) & 0xFFFFu;
-    if (m + 1 < M)
-      *reinterpret_cast<uint32_t*>(Xt + int64_t(k) * ldt + m) = lo | (hi << 16);
-    else
-      Xt[int64_t(k) * ldt + m] = static_cast<uint16_t>(lo);
-  }
+  for (int i = 0; i < 8; ++i) w[i] = tile[8 * j + i][kp];
+  uint4 lo, hi;  // rows k (low halves) and k + 1 (high halves), 8 m each
+  lo.x = __byte_perm(w[0], w[1], 0x5410);
+  lo.y = __byte_perm(w[2], w[3], 0x5410);
+  lo.z = __byte_perm(w[4], w[5], 0x5410);
+  lo.w = __byte_perm(w[6], w[7], 0x5410);
+  hi.x = __byte_perm(w[0], w[1], 0x7632);
+  hi.y = __byte_perm(w[2], w[3], 0x7632);
+  hi.z = __byte_perm(w[4], w[5], 0x7632);
+  hi.w = __byte_perm(w[6], w[7], 0x7632);
+  const int k = k0 + 2 * kp;
+  *reinterpret_cast<uint4*>(Xt + int64_t(k) * ldt + m0 + 8 * j) = lo;
+  *reinterpret_cast<uint4*>(Xt + int64_t(k + 1) * ldt + m0 + 8 * j) = hi;
 }
 
 // ---- run-time GEMM -------------------------------------------------------------------------
@@ -709,7 +722,7 @@ spg_status run(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc
   if (x_layout == SPG_X_MK) {
     uint16_t* ws = static_cast<uint16_t*>(workspace);
     dim3 grid(static_cast<unsigned>((K + 63) / 64), static_cast<unsigned>((M + 63) / 64));
-    transpose_kernel<<<grid, dim3(32, 8), 0, s>>>(static_cast<const uint16_t*>(X), ldx, int(M), int(K), ws, M);
+    transpose_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(X), ldx, int(M), int(K), ws, M);
     xt = ws;
     ldt = M;
   }
@@ -840,7 +853,7 @@ spg_status spgemm_tw_f16_noalloc(const void* X, int64_t ldx, const spg_tw_desc* 
   // every element of the [K][M] region the GEMM reads is written here first,
   // so nothing left in the array by an earlier call is ever read
   dim3 tgrid(static_cast<unsigned>((K + 63) / 64), static_cast<unsigned>((M + 63) / 64));
-  transpose_kernel<<<tgrid, dim3(32, 8), 0, s>>>(static_cast<const uint16_t*>(X), ldx, int(M), int(K), xt, M);
+  transpose_kernel<<<tgrid, 256, 0, s>>>(static_cast<const uint16_t*>(X), ldx, int(M), int(K), xt, M);
   return launch_gemm(xt, M, desc, static_cast<uint16_t*>(Y), ldy, M, s);
 }
 
