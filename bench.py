@@ -156,9 +156,9 @@ class Layer24:
     """Device-resident buffers of one 2:4 layer: `copies` rotating sets of X,
     compressed W, metadata, bias and Y."""
 
-    def __init__(self, spg, d, kind, copies, y_nm=False):
+    def __init__(self, spg, d, kind, copies, y_nm=False, gelu=False):
         import torch
-        self.spg, self.d, self.kind, self.y_nm = spg, d, kind, y_nm
+        self.spg, self.d, self.kind, self.y_nm, self.gelu = spg, d, kind, y_nm, gelu
         dev = torch.device("cuda")
         if kind == "24_s8":
             W = torch.from_numpy(d["W"]).to(dev)
@@ -197,6 +197,8 @@ class Layer24:
             self.spg.spgemm_24_s8(X, self.Wv[i], self.meta[i], self.scale, self.bias[i], Y=Y)
         elif self.y_nm:
             self.spg.spgemm_24_f16_yt(X, self.Wv[i], self.meta[i], self.bias[i], Yt=Y)
+        elif self.gelu:
+            self.spg.spgemm_24_f16_gelu(X, self.Wv[i], self.meta[i], self.bias[i], Y=Y)
         else:
             self.spg.spgemm_24_f16(X, self.Wv[i], self.meta[i], self.bias[i], Y=Y)
 
@@ -261,7 +263,10 @@ def run_ours(args, rank, world, local_rank):
     else:
         if args.y_nm and kind not in ("24_f16", "24_bf16"):
             raise SystemExit("--y-nm applies to the 16-bit 2:4 and tile-wise workloads")
-        layers = [Layer24(spg, d, kind, copies, args.y_nm) for d in inputs]
+        if args.gelu and (kind not in ("24_f16", "24_bf16") or args.y_nm):
+            raise SystemExit("--gelu applies to the 16-bit 2:4 workloads with [M, N] outputs")
+        # --gelu: the activation of an MLP block, fused into its first layer
+        layers = [Layer24(spg, d, kind, copies, args.y_nm, args.gelu and j == 0) for j, d in enumerate(inputs)]
         flops_alg = layer_flops(inputs) / 2.0
         bytes_alg = sum(algorithmic_bytes(d, kind) for d in inputs)
     flops_dense = layer_flops(inputs)
@@ -336,6 +341,7 @@ def run_ours(args, rank, world, local_rank):
     if spg.check_device_error() != 0:
         raise RuntimeError("device error word set during the timed region")
     del g_full, g_rem, g_layer
+    dense = dense_baseline(layers, kind, copies, reps, gstream, stream, args) if args.dense_baseline else None
 
     t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
     if world > 1:
@@ -384,9 +390,63 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roof,
         "e2e": e2e,
         "gpu_launches": args.steps * nl * (2 if (kind == "tw_f16" and not args.x_km) else 1),
+        "dense_cublas": dense,
         "clocks": clocks,
     }
     return out
+
+
+def dense_baseline(layers, kind, copies, reps, gstream, stream, args):
+    """The same layers as dense GEMMs through torch (cuBLAS) on this GPU: dense
+    weights of the same shapes, the same rotating activation buffers, the bias
+    in the GEMM's epilogue (nn.functional.linear), GELU as a separate op where
+    the sparse layer fuses it, and
+    the same graph-replayed timing.  int8 layers use torch._int_mm (int32
+    result, no dequantisation).  Returns per-layer times and the step
+    speedup of the sparse layers over the dense ones."""
+    import torch
+    per_layer = []
+    for L in layers:
+        d = L.d
+        dev = torch.device("cuda")
+        if kind == "24_s8":
+            Wd = [torch.from_numpy(np.ascontiguousarray(d["W"])).to(dev).t() for _ in range(copies)]
+            fn = lambda i, L=L, Wd=Wd: torch._int_mm(L.X[i], Wd[i])
+        else:
+            tdt = L.X[0].dtype
+            if kind == "tw_f16":
+                W = torch.from_numpy(np.ascontiguousarray(d["W"])).to(dev)
+            else:
+                W = Layer24._t(d["W"], tdt, dev)
+            Wd = [W.t()] + [W.clone().t() for _ in range(copies - 1)]
+            bias = getattr(L, "bias", [None])[0]
+            use_gelu = getattr(L, "gelu", False)
+            xs = L.X if not (kind == "tw_f16" and L.x_layout == 1) else [x.t() for x in L.X]
+
+            def fn(i, xs=xs, Wd=Wd, bias=bias, use_gelu=use_gelu):
+                # nn.functional.linear: one cuBLAS(Lt) GEMM with the bias in its epilogue
+                y = torch.nn.functional.linear(xs[i], Wd[i].t(), bias)
+                if use_gelu:
+                    y = torch.nn.functional.gelu(y)
+                return y
+        for i in range(copies):
+            fn(i)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=gstream):
+            outs = [fn(i) for i in range(copies)]
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        per_layer.append(a.elapsed_time(b) / (reps * copies) * 1e3)
+        del g, outs, Wd
+    return {"per_layer_us": per_layer,
+            "what": "torch.nn.functional.linear (+ gelu) / torch._int_mm (cuBLAS), dense weights of the same shapes"}
 
 
 def measure_e2e(spg, layers, kind, args, stream):
@@ -504,6 +564,9 @@ def main():
     ap.add_argument("--y-nm", action="store_true",
                     help="write Y^T [N, M] (the transpose a following tile-wise layer reads, fused into the GEMM)")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--gelu", action="store_true", help="fuse GELU into the first layer (the MLP block's activation)")
+    ap.add_argument("--dense-baseline", action="store_true",
+                    help="also time dense cuBLAS GEMMs of the same shapes and report the speedup")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -533,6 +596,9 @@ def main():
         import torch
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+    if out.get("dense_cublas"):
+        dn = out["dense_cublas"]
+        dn["speedup"] = sum(dn["per_layer_us"]) / sum(out["per_layer_us"])
     if rank == 0:
         print(json.dumps(out), flush=True)
 

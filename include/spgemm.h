@@ -131,6 +131,20 @@ spg_status spgemm_24_f16(const void* X, int64_t ldx, const void* Wv, const uint8
                          spg_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * spgemm_24_f16_gelu  [GPUSQ, Abstract: the 2:4 layers of a vision
+ * transformer; the activation between the two layers of its MLP block]
+ *
+ * spgemm_24_f16 with the activation fused into the epilogue:
+ *   Y[m][n] = round( GELU( sum_k X[m][k] * Wm[n][k] (+ bias[n]) ) )
+ * with GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt(2))) evaluated in fp32
+ * after the fp32 bias add, then one round-to-nearest-even to `dtype`.
+ * Same arguments and limits as spgemm_24_f16.
+ * ------------------------------------------------------------------------- */
+spg_status spgemm_24_f16_gelu(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,
+                              void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, spg_dtype dtype,
+                              spg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * spgemm_24_f16_yt  [GPUSQ, Abstract; TW, slide "Transpose": the transpose
  * the next tile-wise layer needs, fused into the producing layer]
  *

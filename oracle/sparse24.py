@@ -132,6 +132,20 @@ def gemm_24_ref(X, Wv, meta, bias, dtype: str, rows=None) -> np.ndarray:
     return Y
 
 
+def gelu_ref(Y: np.ndarray) -> np.ndarray:
+    """GELU(y) = y * Phi(y) = 0.5 y (1 + erf(y / sqrt(2))) in fp64.
+
+    The activation between the two linear layers of the MLP block of the
+    vision transformers the 2:4 scheme compresses ("Boost Vision Transformer
+    with GPU-Friendly Sparsity and Quantization", Abstract: ViT models); the
+    pages do not spell it out, so the exact (erf) form of the ViT MLP is used.
+    erf is scipy's fp64 routine, a library step.
+    """
+    from scipy.special import erf
+    Y = np.asarray(Y, dtype=np.float64)
+    return 0.5 * Y * (1.0 + erf(Y / np.sqrt(2.0)))
+
+
 def gemm_24_s8_ref(X, Wv, meta, rows=None) -> np.ndarray:
     """Exact int8 2:4 accumulator acc[m, n] = sum_k x[m,k] * wm[n,k] (int64).
 

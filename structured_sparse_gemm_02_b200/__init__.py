@@ -48,6 +48,7 @@ SIGNATURES = {
     "sparse_prune_24": (ctypes.c_int, [_p, _i64, _p, _i64, _i64, _i64, ctypes.c_int, _p]),
     "sparse_compress_24": (ctypes.c_int, [_p, _i64, _p, _p, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_f16": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
+    "spgemm_24_f16_gelu": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_f16_yt": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_s8": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _p, _i64, ctypes.c_int, _i64, _i64, _i64, _p]),
     "tw_query_sizes": (ctypes.c_int, [_i64, _i64, _i32, _i64, ctypes.POINTER(_i32), ctypes.POINTER(SpgTwSizes)]),
@@ -157,6 +158,19 @@ def spgemm_24_f16(X, Wv, meta, bias=None, Y=None, stream=None):
     if Y is None:
         Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
     _check("spgemm_24_f16", lib().spgemm_24_f16(
+        _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(bias), _ptr(Y), Y.stride(0), M, N, K,
+        _dtype_code(X), _stream(stream)))
+    return Y
+
+
+def spgemm_24_f16_gelu(X, Wv, meta, bias=None, Y=None, stream=None):
+    """Y [M, N] = GELU(X [M, K] . decompress(Wv, meta)^T (+ bias)), fp16 or bf16."""
+    import torch
+    M, K = X.shape
+    N = Wv.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    _check("spgemm_24_f16_gelu", lib().spgemm_24_f16_gelu(
         _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(bias), _ptr(Y), Y.stride(0), M, N, K,
         _dtype_code(X), _stream(stream)))
     return Y

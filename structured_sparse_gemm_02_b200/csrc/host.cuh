@@ -30,6 +30,25 @@ bool make_tmap_2d_swz(CUtensorMap* map, const void* base, int esize, uint64_t co
 
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Launch `kernel` on `stream` with programmatic stream serialisation allowed
+// (the kernel calls griddep_launch_dependents / griddep_wait, sm100.cuh), so
+// its launch and prologue overlap the end of the previous kernel.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 inline spg_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? SPG_OK : SPG_ERR_CUDA;
 }

@@ -37,6 +37,19 @@ __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// ---- programmatic dependent launch ---------------------------------------------
+// The kernels below are launched with programmatic stream serialisation: the
+// next kernel of the stream may start launching once every block of this one
+// has called griddep_launch_dependents() (or exited), and griddep_wait()
+// returns once the previous kernel of the stream has completed with all its
+// memory operations visible.  Without a programmatic dependency both return
+// at once.  A kernel calls griddep_wait() before it touches global memory that
+// another kernel may write or read.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---- mbarrier ----------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count));

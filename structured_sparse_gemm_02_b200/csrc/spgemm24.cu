@@ -39,7 +39,14 @@ namespace gemm24 {
 // Output kinds: Y [M][N] in fp16 / bf16 / int32, or the transpose Y^T [N][M]
 // in fp16 / bf16 (the layout a following tile-wise layer reads as its
 // activations, so that layer needs no transpose).
-enum OutKind { OUT_F16 = 0, OUT_BF16 = 1, OUT_S32 = 2, OUT_F16_T = 3, OUT_BF16_T = 4 };
+// GELU kinds: Y [M][N] = GELU(acc + bias) in fp16 / bf16 (the activation
+// between the two layers of a transformer MLP block, fused into the first).
+enum OutKind { OUT_F16 = 0, OUT_BF16 = 1, OUT_S32 = 2, OUT_F16_T = 3, OUT_BF16_T = 4, OUT_F16_G = 5, OUT_BF16_G = 6 };
+__host__ __device__ constexpr bool out_bf16(int k) { return k == OUT_BF16 || k == OUT_BF16_T || k == OUT_BF16_G; }
+__host__ __device__ constexpr bool out_gelu(int k) { return k == OUT_F16_G || k == OUT_BF16_G; }
+
+// GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), in fp32.
+__device__ __forceinline__ float gelu_f32(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
 
 // Pair tile: 256 weight rows (128 per CTA of the cluster pair) x BN rows of X
 // (BN/2 loaded by each CTA).  STAGES is the deepest operand ring that fits.
@@ -55,7 +62,7 @@ struct Cfg {
   static constexpr int MCOLS = kInt8 ? 8 : 4;          // TMEM columns of metadata per stage
   static constexpr int OUT_ES = OUT == OUT_S32 ? 4 : 2;
   static constexpr bool YT = OUT == OUT_F16_T || OUT == OUT_BF16_T;  // Y^T: stored from registers
-  static constexpr bool OUT_BF = OUT == OUT_BF16 || OUT == OUT_BF16_T;
+  static constexpr bool OUT_BF = out_bf16(OUT);
   // staging per epilogue warp: 16-bit outputs double-buffer a 4 KB box per warp
   // pair (2 KB per warp and buffer); int32 outputs one 4 KB box per warp
   static constexpr int EPI_BUF = OUT_ES == 2 ? 2 * 2048 : 4096;
@@ -148,10 +155,13 @@ __device__ __forceinline__ uint32_t convert_out(uint32_t acc, float badd, float 
     float v = __fmul_rn(__int2float_rn(static_cast<int>(acc)), sc);
     if (has_bias) v = __fadd_rn(v, badd);
     return __half_as_ushort(__float2half_rn(v));
-  } else if constexpr (OUT == OUT_BF16 || OUT == OUT_BF16_T) {
-    return __bfloat16_as_ushort(__float2bfloat16_rn(__fadd_rn(__uint_as_float(acc), badd)));
   } else {
-    return __half_as_ushort(__float2half_rn(__fadd_rn(__uint_as_float(acc), badd)));
+    float v = __fadd_rn(__uint_as_float(acc), badd);
+    if constexpr (out_gelu(OUT)) v = gelu_f32(v);
+    if constexpr (out_bf16(OUT))
+      return __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    else
+      return __half_as_ushort(__float2half_rn(v));
   }
 }
 
@@ -171,9 +181,13 @@ __device__ __forceinline__ uint32_t convert_pair16(uint32_t a0, uint32_t a1, flo
   } else {
     v0 = __fadd_rn(__uint_as_float(a0), badd);
     v1 = __fadd_rn(__uint_as_float(a1), badd);
+    if constexpr (out_gelu(OUT)) {
+      v0 = gelu_f32(v0);
+      v1 = gelu_f32(v1);
+    }
   }
   uint32_t w;
-  if constexpr (OUT == OUT_BF16 || OUT == OUT_BF16_T)
+  if constexpr (out_bf16(OUT))
     asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(v1), "f"(v0));
   else
     asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(v1), "f"(v0));
@@ -273,6 +287,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   cluster_sync();  // barriers of both CTAs initialised, tensor memory allocated
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  griddep_launch_dependents();
+  griddep_wait();  // the previous kernel's writes (X, or readers of Y) are complete
   // the leader's barriers as seen from either CTA of the pair
   const uint32_t full_l = mapa_shared(smem_addr(full), 0);
   const uint32_t meta_full_l = mapa_shared(smem_addr(meta_full), 0);
@@ -625,8 +641,9 @@ spg_status launch(const void* X, int64_t ldx, const void* Wv, const uint8_t* met
   const int64_t pairs_max = resident_pairs(reinterpret_cast<const void*>(kern), C::SMEM, C::THREADS);
   if (pairs_max <= 0) return SPG_ERR_CUDA;
   const int pairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
-  kern<<<2 * pairs, C::THREADS, C::SMEM, stream>>>(tmA, tmB, tmE, tmY, Y, ldy, bias, scale, static_cast<int>(M),
-                                            static_cast<int>(N), static_cast<int>(K), err);
+  if (launch_pdl(kern, dim3(2 * pairs), dim3(C::THREADS), C::SMEM, stream, tmA, tmB, tmE, tmY, Y, ldy, bias, scale, static_cast<int>(M),
+                                            static_cast<int>(N), static_cast<int>(K), err) != cudaSuccess)
+    return SPG_ERR_CUDA;
   return launch_status();
 }
 
@@ -671,6 +688,23 @@ spg_status spgemm_24_f16(const void* X, int64_t ldx, const void* Wv, const uint8
   auto s = reinterpret_cast<cudaStream_t>(stream);
   if (dtype == SPG_F16) return dispatch<false, false, OUT_F16>(X, ldx, Wv, meta, bias, nullptr, Y, ldy, M, N, K, s);
   return dispatch<false, true, OUT_BF16>(X, ldx, Wv, meta, bias, nullptr, Y, ldy, M, N, K, s);
+}
+
+spg_status spgemm_24_f16_gelu(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,
+                              void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, spg_dtype dtype,
+                              spg_stream_t stream) {
+  using namespace spg;
+  using namespace spg::gemm24;
+  if (dtype != SPG_F16 && dtype != SPG_BF16) return SPG_ERR_INVALID_ARG;
+  spg_status st = validate_common(X, ldx, Wv, meta, Y, ldy, M, N, K, 2, 2, 128);
+  if (st != SPG_OK) return st;
+  if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;
+  st = check_device();
+  if (st != SPG_OK) return st;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  if (dtype == SPG_F16)
+    return dispatch<false, false, OUT_F16_G>(X, ldx, Wv, meta, bias, nullptr, Y, ldy, M, N, K, s);
+  return dispatch<false, true, OUT_BF16_G>(X, ldx, Wv, meta, bias, nullptr, Y, ldy, M, N, K, s);
 }
 
 spg_status spgemm_24_f16_yt(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,

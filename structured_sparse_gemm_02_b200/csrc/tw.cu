@@ -192,6 +192,8 @@ __global__ void gather_wc_kernel(const uint16_t* __restrict__ W, int64_t ldw, in
 __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restrict__ X, int64_t ldx, int M, int K,
                                                         uint16_t* __restrict__ Xt, int64_t ldt) {
   __shared__ uint32_t tile[64][33];  // [m][k pair]
+  griddep_launch_dependents();
+  griddep_wait();
   const int m0 = blockIdx.y * 64, k0 = blockIdx.x * 64;
   const int t = threadIdx.x;
   {
@@ -334,6 +336,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  griddep_launch_dependents();
+  griddep_wait();  // the previous kernel's writes (Xt, or readers of Y) are complete
 
   if (warp < 2) {
     // ---------------- loads ----------------
@@ -690,9 +694,10 @@ spg_status launch_gemm(const uint16_t* xt, int64_t ldt, const spg_tw_desc* desc,
   if (!smem_attr_set()) return SPG_ERR_CUDA;
   const int64_t units = int64_t(desc->T) * ((M + BN - 1) / BN);
   const int grid = static_cast<int>(units < sm_count() ? units : sm_count());
-  tw_gemm_kernel<<<grid, THREADS, SMEM, s>>>(tmWc, tmY64, tmY8, xt, ldt, Y, ldy, vec_ok, y_nm ? 1 : 0, int(M),
+  if (launch_pdl(tw_gemm_kernel, dim3(grid), dim3(THREADS), SMEM, s, tmWc, tmY64, tmY8, xt, ldt, Y, ldy, vec_ok, y_nm ? 1 : 0, int(M),
                                               int(desc->Nk), desc->T,
-                                         desc->offsetn, desc->tile_n0, desc->tile_kofs, desc->offsetk, err);
+                                         desc->offsetn, desc->tile_n0, desc->tile_kofs, desc->offsetk, err) != cudaSuccess)
+    return SPG_ERR_CUDA;
   return launch_status();
 }
 
@@ -722,7 +727,9 @@ spg_status run(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc
   if (x_layout == SPG_X_MK) {
     uint16_t* ws = static_cast<uint16_t*>(workspace);
     dim3 grid(static_cast<unsigned>((K + 63) / 64), static_cast<unsigned>((M + 63) / 64));
-    transpose_kernel<<<grid, 256, 0, s>>>(static_cast<const uint16_t*>(X), ldx, int(M), int(K), ws, M);
+    if (launch_pdl(transpose_kernel, grid, dim3(256), 0, s, static_cast<const uint16_t*>(X), ldx, int(M), int(K), ws,
+                   M) != cudaSuccess)
+      return SPG_ERR_CUDA;
     xt = ws;
     ldt = M;
   }
@@ -853,7 +860,9 @@ spg_status spgemm_tw_f16_noalloc(const void* X, int64_t ldx, const spg_tw_desc* 
   // every element of the [K][M] region the GEMM reads is written here first,
   // so nothing left in the array by an earlier call is ever read
   dim3 tgrid(static_cast<unsigned>((K + 63) / 64), static_cast<unsigned>((M + 63) / 64));
-  transpose_kernel<<<tgrid, 256, 0, s>>>(static_cast<const uint16_t*>(X), ldx, int(M), int(K), xt, M);
+  if (launch_pdl(transpose_kernel, tgrid, dim3(256), 0, s, static_cast<const uint16_t*>(X), ldx, int(M), int(K), xt,
+                 M) != cudaSuccess)
+    return SPG_ERR_CUDA;
   return launch_gemm(xt, M, desc, static_cast<uint16_t*>(Y), ldy, M, s);
 }
 

@@ -200,3 +200,36 @@ def test_bf16_decode_and_prefill_sampled(spg):
     ref = s24.gemm_24_ref(dp["X"], Wv, meta, None, "bf16", rows=rows)
     rep = compare.check_close(s24.to_f64(Yp[rows], "bf16"), ref, dp["K"])
     assert rep["ok"], rep
+
+
+@pytest.mark.parametrize("kind", ["f16", "bf16"])
+@pytest.mark.parametrize("M,N,K", [(17, 129, 384), (300, 200, 640), (2000, 520, 256)])
+def test_gelu_epilogue_ragged(spg, kind, M, N, K):
+    """Y = GELU(X . Wm^T + bias) fused in the epilogue, against the fp64 oracle."""
+    import torch
+    rng = np.random.default_rng(7 * M + N)
+    cv = (lambda a: a.astype(np.float16)) if kind == "f16" else gen.f32_to_bf16_bits
+    X = cv(rng.standard_normal((M, K)).astype(np.float32))
+    W = cv((rng.standard_normal((N, K)) * 0.05).astype(np.float32))
+    b = cv((rng.standard_normal(N) * 0.1).astype(np.float32))
+    Xd, Wd, bd = to_dev(X, kind), to_dev(W, kind), to_dev(b, kind)
+    Wv, meta = spg.sparse_compress_24(Wd)
+    Ybuf = torch.empty((M, (N + 7) // 8 * 8), dtype=Xd.dtype, device="cuda")
+    Y = spg.spgemm_24_f16_gelu(Xd, Wv, meta, bd, Y=Ybuf[:, :N])
+    assert spg.check_device_error() == 0
+    got = s24.to_f64(to_host(Y.contiguous(), kind), kind)
+    ref = s24.gelu_ref(s24.gemm_24_ref(X, *s24.compress_24(W, kind), b, kind))
+    rep = compare.check_close(got, ref, K)
+    assert rep["ok"], rep
+
+
+def test_gelu_epilogue_vitb_fc1_sampled(spg):
+    import torch
+    d = gen.make_inputs("vitb_mlp_f16", layers=["fc1"])[0]
+    Wv, meta = spg.sparse_compress_24(torch.from_numpy(d["W"]).cuda())
+    Y = spg.spgemm_24_f16_gelu(torch.from_numpy(d["X"]).cuda(), Wv, meta, torch.from_numpy(d["bias"]).cuda())
+    assert spg.check_device_error() == 0
+    rows = np.unique(np.concatenate([np.arange(0, d["M"], 97), [d["M"] - 1]]))
+    ref = s24.gelu_ref(s24.gemm_24_ref(d["X"], *s24.compress_24(d["W"], "f16"), d["bias"], "f16", rows=rows))
+    rep = compare.check_close(Y.cpu().numpy()[rows].astype(np.float64), ref, d["K"])
+    assert rep["ok"], rep

@@ -178,3 +178,21 @@ def test_dequant_exact_cases_and_rounding_bound():
     exact = acc[0].astype(np.float64) * scale.astype(np.float64)
     ulp = np.spacing(np.abs(exact).astype(np.float16)).astype(np.float64)
     assert (np.abs(y - exact) <= 0.5 * ulp + np.abs(exact) * 2 ** -23).all()
+
+
+def test_gelu_textbook_values_and_symmetry():
+    """GELU(y) = y * Phi(y), pinned by standard-normal table values and the
+    identity Phi(y) + Phi(-y) = 1 (so GELU(y) - GELU(-y) = y)."""
+    import numpy as np
+    from oracle import sparse24 as s24
+    table = {0.0: 0.5, 1.0: 0.8413447460685429, 2.0: 0.9772498680518208, -1.0: 0.15865525393145707,
+             0.5: 0.6914624612740131, -2.5: 0.006209665325776132}
+    y = np.array(sorted(table))
+    got = s24.gelu_ref(y)
+    want = y * np.array([table[v] for v in y])
+    assert np.allclose(got, want, rtol=1e-14, atol=1e-15)
+    grid = np.linspace(-8, 8, 1601)
+    assert np.allclose(s24.gelu_ref(grid) - s24.gelu_ref(-grid), grid, rtol=0, atol=1e-14)
+    assert s24.gelu_ref(np.array([0.0]))[0] == 0.0
+    assert abs(s24.gelu_ref(np.array([10.0]))[0] - 10.0) < 1e-12
+    assert abs(s24.gelu_ref(np.array([-10.0]))[0]) < 1e-12
