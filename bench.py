@@ -82,7 +82,9 @@ def algorithmic_bytes(d, kind):
     """X read once, compressed W + metadata (+bias/scale) read once, Y written once."""
     M, N, K = d["M"], d["N"], d["K"]
     if kind == "24_s8":
-        return M * K + N * K // 2 + N * K // 8 + 4 * N + 2 * M * N
+        bias = 2 * N if d.get("bias") is not None else 0
+        out = M * N if d.get("qscale") is not None else 2 * M * N
+        return M * K + N * K // 2 + N * K // 8 + 4 * N + bias + out
     b = 2 * N if d.get("bias") is not None else 0
     return 2 * M * K + 2 * N * K // 2 + N * K // 8 + b + 2 * M * N
 
@@ -160,11 +162,12 @@ class Layer24:
         import torch
         self.spg, self.d, self.kind, self.y_nm, self.gelu = spg, d, kind, y_nm, gelu
         dev = torch.device("cuda")
+        self.qscale = d.get("qscale")   # int8 output for the next int8 layer (GELU, quantise)
         if kind == "24_s8":
             W = torch.from_numpy(d["W"]).to(dev)
-            X = torch.from_numpy(d["X"]).to(dev)
+            X = torch.from_numpy(d["X"]).to(dev) if d["X"] is not None else None
             self.scale = torch.from_numpy(d["scale"]).to(dev)
-            self.out_dtype = torch.float16
+            self.out_dtype = torch.int8 if self.qscale is not None else torch.float16
         else:
             tdt = torch.bfloat16 if kind == "24_bf16" else torch.float16
             W = self._t(d["W"], tdt, dev)
@@ -174,7 +177,8 @@ class Layer24:
         bias = self._t(d["bias"], self.out_dtype, dev) if d.get("bias") is not None else None
         Wv, meta = spg.sparse_compress_24(W)
         del W
-        self.X = [X] + [X.clone() for _ in range(copies - 1)]
+        # X is None for a layer whose input is the previous layer's output (linked by the caller)
+        self.X = [X] + [X.clone() for _ in range(copies - 1)] if X is not None else None
         self.Wv = [Wv] + [Wv.clone() for _ in range(copies - 1)]
         self.meta = [meta] + [meta.clone() for _ in range(copies - 1)]
         self.bias = [bias] + [bias.clone() if bias is not None else None for _ in range(copies - 1)]
@@ -193,7 +197,10 @@ class Layer24:
     def run(self, i, X=None, Y=None):
         X = self.X[i] if X is None else X
         Y = self.Y[i] if Y is None else Y
-        if self.kind == "24_s8":
+        if self.kind == "24_s8" and self.qscale is not None:
+            self.spg.spgemm_24_s8_q(X, self.Wv[i], self.meta[i], self.scale, self.bias[i], self.qscale,
+                                    self.spg.SPG_ACT_GELU, Yq=Y)
+        elif self.kind == "24_s8":
             self.spg.spgemm_24_s8(X, self.Wv[i], self.meta[i], self.scale, self.bias[i], Y=Y)
         elif self.y_nm:
             self.spg.spgemm_24_f16_yt(X, self.Wv[i], self.meta[i], self.bias[i], Yt=Y)
@@ -267,6 +274,9 @@ def run_ours(args, rank, world, local_rank):
             raise SystemExit("--gelu applies to the 16-bit 2:4 workloads with [M, N] outputs")
         # --gelu: the activation of an MLP block, fused into its first layer
         layers = [Layer24(spg, d, kind, copies, args.y_nm, args.gelu and j == 0) for j, d in enumerate(inputs)]
+        for j, L in enumerate(layers):
+            if L.X is None:        # a chained layer reads the previous layer's output buffers
+                L.X = layers[j - 1].Y
         flops_alg = layer_flops(inputs) / 2.0
         bytes_alg = sum(algorithmic_bytes(d, kind) for d in inputs)
     flops_dense = layer_flops(inputs)
@@ -453,17 +463,21 @@ def measure_e2e(spg, layers, kind, args, stream):
     import torch
     steps = max(3, min(args.e2e_steps, args.steps))
     hx, hy = [], []
-    for L in layers:
-        hx.append(L.X[0].cpu().pin_memory())
-        hy.append(torch.empty(L.Y[0].shape, dtype=L.Y[0].dtype).pin_memory())
-    bi = sum(t.numel() * t.element_size() for t in hx)
-    bo = sum(t.numel() * t.element_size() for t in hy)
+    for j, L in enumerate(layers):
+        chained_in = j > 0 and L.X is layers[j - 1].Y
+        consumed = j + 1 < len(layers) and layers[j + 1].X is L.Y
+        hx.append(None if chained_in else L.X[0].cpu().pin_memory())
+        hy.append(None if consumed else torch.empty(L.Y[0].shape, dtype=L.Y[0].dtype).pin_memory())
+    bi = sum(t.numel() * t.element_size() for t in hx if t is not None)
+    bo = sum(t.numel() * t.element_size() for t in hy if t is not None)
 
     def once():
         for L, x, y in zip(layers, hx, hy):
-            L.X[0].copy_(x, non_blocking=True)
+            if x is not None:
+                L.X[0].copy_(x, non_blocking=True)
             L.run(0)
-            y.copy_(L.Y[0], non_blocking=True)
+            if y is not None:
+                y.copy_(L.Y[0], non_blocking=True)
 
     once()
     torch.cuda.synchronize()
@@ -486,6 +500,7 @@ def oracle_step(inputs, kind, rows_frac=1.0):
     """Run the oracle over (a row sample of) every layer; returns dense-eq FLOPs computed."""
     from oracle import sparse24 as s24, tilewise as tw
     flops = 0.0
+    prev = None
     for d in inputs:
         rows = None
         M = d["M"]
@@ -497,8 +512,14 @@ def oracle_step(inputs, kind, rows_frac=1.0):
             tw.tw_gemm_ref(d["X"], r, rows=rows)
         elif kind == "24_s8":
             Wv, meta = s24.compress_24(d["W"], "s8")
-            acc = s24.gemm_24_s8_ref(d["X"], Wv, meta, rows=rows)
-            s24.dequant_s8(acc, d["scale"])
+            if d["X"] is None:          # chained: the previous layer's int8 output (same rows)
+                acc = s24.gemm_24_s8_ref(prev, Wv, meta)
+            else:
+                acc = s24.gemm_24_s8_ref(d["X"], Wv, meta, rows=rows)
+            if d.get("qscale") is not None:
+                prev = s24.quantize_s8(acc, d["scale"], d.get("bias"), d["qscale"], True)
+            else:
+                s24.dequant_s8(acc, d["scale"], d.get("bias"))
         else:
             k = DTYPE_NAME[kind]
             Wv, meta = s24.compress_24(d["W"], k)

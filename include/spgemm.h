@@ -54,6 +54,7 @@ typedef enum { SPG_F16 = 0, SPG_BF16 = 1, SPG_S8 = 2 } spg_dtype;
 
 enum { SPG_OUT_F16 = 0, SPG_OUT_S32 = 1 };  /* spgemm_24_s8 output modes */
 enum { SPG_X_MK = 0, SPG_X_KM = 1 };        /* spgemm_tw_f16 activation layouts */
+enum { SPG_ACT_NONE = 0, SPG_ACT_GELU = 1 }; /* spgemm_24_s8_q activations */
 
 /* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
 int spg_version(void);
@@ -178,6 +179,31 @@ spg_status spgemm_24_f16_yt(const void* X, int64_t ldx, const void* Wv, const ui
 spg_status spgemm_24_s8(const int8_t* X, int64_t ldx, const int8_t* Wv, const uint8_t* meta, const float* scale,
                         const void* bias, void* Y, int64_t ldy, int out_mode, int64_t M, int64_t N, int64_t K,
                         spg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * spgemm_24_s8_q  [GPUSQ, Abstract: the fixed-point (int8) 2:4 model; the
+ * int8 activations of the next layer produced by this layer's epilogue]
+ *
+ * acc as spgemm_24_s8, then per element, in fp32 with one round-to-nearest-
+ * even per operation and no fused multiply-add:
+ *   v = fp32(acc) * scale[n]  [ + fp32(bias[n]) ]
+ *   act SPG_ACT_GELU: v = GELU(v) = (0.5 v) (1 + erf(v * 0.70710677)), with
+ *     erf(u) = sign(u) (1 - r) (Abramowitz & Stegun 7.1.28, |error| <= 3e-7):
+ *     a = min(|u|, 4); p = ((((((a6 a + a5) a + a4) a + a3) a + a2) a + a1) a)
+ *     + 1 with a1..a6 = 0.0705230784, 0.0422820123, 0.0092705272,
+ *     0.0001520143, 0.0002765672, 0.0000430638; p^16 by four squarings;
+ *     r = 1 / p^16 by three Newton steps r = r (2 - p^16 r) from the fp32
+ *     whose bits are 0x7EF00000 - bits(p^16)
+ *   Yq[m][n] (int8) = clamp( rne( v * qscale ), -127, 127 )
+ * qscale is the reciprocal of the next layer's activation scale (that scale is
+ * folded into the next layer's scale[]).  The fixed operation order makes the
+ * int8 codes reproducible bit for bit on the host.
+ *   X, Wv, meta, scale, bias as spgemm_24_s8; Yq int8 [M, N], pitch ldy
+ *   (bytes, a multiple of 16), 16-byte aligned; 0 < qscale < 3e38.
+ * ------------------------------------------------------------------------- */
+spg_status spgemm_24_s8_q(const int8_t* X, int64_t ldx, const int8_t* Wv, const uint8_t* meta, const float* scale,
+                          const void* bias, float qscale, int act, int8_t* Yq, int64_t ldy, int64_t M, int64_t N,
+                          int64_t K, spg_stream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Tile-wise sparsity  [TW, slides "Tile-Wise Sparsity", "Re-organize",

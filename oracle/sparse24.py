@@ -175,3 +175,61 @@ def dequant_s8(acc: np.ndarray, scale: np.ndarray, bias=None) -> np.ndarray:
     if bias is not None:
         v = (v + np.asarray(bias, dtype=np.float16).astype(np.float32)[None, :]).astype(np.float32)
     return v.astype(np.float16)
+
+
+# ---- int8 activations for the next int8 layer ---------------------------------------------
+# Coefficients of Abramowitz & Stegun 7.1.28: erf(a) = 1 - 1/(1 + a1 a + ... + a6 a^6)^16
+# for a >= 0, with |error| <= 3e-7.
+AS_ERF_A = (0.0705230784, 0.0422820123, 0.0092705272, 0.0001520143, 0.0002765672, 0.0000430638)
+
+
+def erf_as_f32(u: np.ndarray) -> np.ndarray:
+    """erf by A&S 7.1.28 in fp32, every operation one round-to-nearest-even:
+    a = min(|u|, 4) (at 4 the value is already 1.0 in fp32);
+    p = ((((((a6 a + a5) a + a4) a + a3) a + a2) a + a1) a) + 1;
+    p^16 by four squarings; r = 1 / p^16 by three Newton steps
+    r = r (2 - p^16 r) from the seed with bits 0x7EF00000 - bits(p^16);
+    erf = sign(u) (1 - r)."""
+    f = np.float32
+    u = np.asarray(u, dtype=np.float32)
+    a = np.minimum(np.abs(u), f(4.0))
+    a1, a2, a3, a4, a5, a6 = (f(c) for c in AS_ERF_A)
+    h = np.full_like(a, a6)
+    for c in (a5, a4, a3, a2, a1):
+        h = (h * a).astype(np.float32)
+        h = (h + c).astype(np.float32)
+    p = ((h * a).astype(np.float32) + f(1.0)).astype(np.float32)
+    p2 = (p * p).astype(np.float32)
+    p4 = (p2 * p2).astype(np.float32)
+    p8 = (p4 * p4).astype(np.float32)
+    p16 = (p8 * p8).astype(np.float32)
+    r = (np.uint32(0x7EF00000) - p16.view(np.uint32)).view(np.float32)
+    for _ in range(3):
+        t = (p16 * r).astype(np.float32)
+        t = (f(2.0) - t).astype(np.float32)
+        r = (r * t).astype(np.float32)
+    e = (f(1.0) - r).astype(np.float32)
+    return np.where(u < 0, -e, e).astype(np.float32)
+
+
+def gelu_as_f32(v: np.ndarray) -> np.ndarray:
+    """GELU(v) = (0.5 v) (1 + erf(v * 0.70710677)) in fp32 with erf_as_f32, each
+    operation rounded once, in that order."""
+    f = np.float32
+    v = np.asarray(v, dtype=np.float32)
+    u = (v * f(0.70710677)).astype(np.float32)
+    return ((f(0.5) * v).astype(np.float32) * (f(1.0) + erf_as_f32(u)).astype(np.float32)).astype(np.float32)
+
+
+def quantize_s8(acc: np.ndarray, scale: np.ndarray, bias, qscale: float, gelu: bool) -> np.ndarray:
+    """Epilogue that feeds the next int8 layer: v = fp32(acc) *rn scale[n]
+    [+rn fp32(bias[n])], [v = GELU(v)], q = clamp(rne(v *rn qscale), -127, 127)."""
+    v = np.asarray(acc).astype(np.float32)
+    v = (v * np.asarray(scale, dtype=np.float32)[None, :]).astype(np.float32)
+    if bias is not None:
+        v = (v + np.asarray(bias, dtype=np.float16).astype(np.float32)[None, :]).astype(np.float32)
+    if gelu:
+        v = gelu_as_f32(v)
+    t = (v * np.float32(qscale)).astype(np.float32)
+    return np.clip(np.rint(t), -127, 127).astype(np.int8)
+

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libspgemm.so")
 SPG_F16, SPG_BF16, SPG_S8 = 0, 1, 2
 SPG_OUT_F16, SPG_OUT_S32 = 0, 1
 SPG_X_MK, SPG_X_KM = 0, 1
+SPG_ACT_NONE, SPG_ACT_GELU = 0, 1
 
 _STATUS = {
     0: "SPG_OK", 1: "SPG_ERR_INVALID_ARG", 2: "SPG_ERR_UNSUPPORTED_SHAPE", 3: "SPG_ERR_MISALIGNED",
@@ -51,6 +52,8 @@ SIGNATURES = {
     "spgemm_24_f16_gelu": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_f16_yt": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_s8": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _p, _i64, ctypes.c_int, _i64, _i64, _i64, _p]),
+    "spgemm_24_s8_q": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, ctypes.c_float, ctypes.c_int, _p, _i64, _i64, _i64,
+                                      _i64, _p]),
     "tw_query_sizes": (ctypes.c_int, [_i64, _i64, _i32, _i64, ctypes.POINTER(_i32), ctypes.POINTER(SpgTwSizes)]),
     "tw_reorganize": (ctypes.c_int, [_p, _i64, _i64, ctypes.POINTER(_i32), ctypes.POINTER(SpgTwDesc), _p, _sz,
                                      _p]),
@@ -201,6 +204,20 @@ def spgemm_24_s8(X, Wv, meta, scale=None, bias=None, Y=None, out_mode=SPG_OUT_F1
         _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(scale), _ptr(bias), _ptr(Y), Y.stride(0),
         out_mode, M, N, K, _stream(stream)))
     return Y
+
+
+def spgemm_24_s8_q(X, Wv, meta, scale, bias=None, qscale=1.0, act=SPG_ACT_NONE, Yq=None, stream=None):
+    """int8 2:4 layer whose epilogue emits int8 activations for the next int8 layer:
+    Yq = clamp(rne(act(fp32(acc) * scale (+ bias)) * qscale), -127, 127)."""
+    import torch
+    M, K = X.shape
+    N = Wv.shape[0]
+    if Yq is None:
+        Yq = torch.empty((M, N), dtype=torch.int8, device=X.device)
+    _check("spgemm_24_s8_q", lib().spgemm_24_s8_q(
+        _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(scale), _ptr(bias), float(qscale), int(act), _ptr(Yq),
+        Yq.stride(0), M, N, K, _stream(stream)))
+    return Yq
 
 
 class TwDesc:

@@ -28,6 +28,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <cstring>
 
 #include "host.cuh"
 #include "sm100.cuh"
@@ -41,12 +42,50 @@ namespace gemm24 {
 // activations, so that layer needs no transpose).
 // GELU kinds: Y [M][N] = GELU(acc + bias) in fp16 / bf16 (the activation
 // between the two layers of a transformer MLP block, fused into the first).
-enum OutKind { OUT_F16 = 0, OUT_BF16 = 1, OUT_S32 = 2, OUT_F16_T = 3, OUT_BF16_T = 4, OUT_F16_G = 5, OUT_BF16_G = 6 };
+// Quantised kinds (int8 inputs only): Y [M][N] int8 = clamp(rne(v * qscale))
+// with v the dequantised value, optionally through GELU first: the int8
+// activations of the next 2:4 int8 layer.
+enum OutKind {
+  OUT_F16 = 0, OUT_BF16 = 1, OUT_S32 = 2, OUT_F16_T = 3, OUT_BF16_T = 4, OUT_F16_G = 5, OUT_BF16_G = 6,
+  OUT_S8Q = 7, OUT_S8QG = 8
+};
 __host__ __device__ constexpr bool out_bf16(int k) { return k == OUT_BF16 || k == OUT_BF16_T || k == OUT_BF16_G; }
-__host__ __device__ constexpr bool out_gelu(int k) { return k == OUT_F16_G || k == OUT_BF16_G; }
+__host__ __device__ constexpr bool out_gelu(int k) { return k == OUT_F16_G || k == OUT_BF16_G || k == OUT_S8QG; }
+__host__ __device__ constexpr bool out_s8(int k) { return k == OUT_S8Q || k == OUT_S8QG; }
 
 // GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), in fp32.
 __device__ __forceinline__ float gelu_f32(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
+
+// GELU for the quantised path, where the rounded result decides an integer
+// code and must be reproducible bit for bit on the host: erf from
+// Abramowitz & Stegun 7.1.28, erf(a) = 1 - 1 / (1 + a1 a + ... + a6 a^6)^16
+// for a >= 0 (|error| <= 3e-7), odd extension.  Every operation is one fp32
+// round-to-nearest-even in the order written, no fused multiply-add:
+//  * a = min(|u|, 4): at 4 the result is already 1.0f, so p^16 stays finite;
+//  * 1 / p^16 by three Newton steps r = r (2 - x r) from the seed whose bits
+//    are 0x7EF00000 - bits(x) (exponent flipped, within 6.25 %): relative
+//    error about 1.5e-7 and no division.
+__device__ __forceinline__ float gelu_as_f32(float v) {
+  const float u = __fmul_rn(v, 0.70710677f);
+  const float a = fminf(fabsf(u), 4.0f);
+  float h = 0.0000430638f;
+  h = __fadd_rn(__fmul_rn(h, a), 0.0002765672f);
+  h = __fadd_rn(__fmul_rn(h, a), 0.0001520143f);
+  h = __fadd_rn(__fmul_rn(h, a), 0.0092705272f);
+  h = __fadd_rn(__fmul_rn(h, a), 0.0422820123f);
+  h = __fadd_rn(__fmul_rn(h, a), 0.0705230784f);
+  const float p = __fadd_rn(__fmul_rn(h, a), 1.0f);
+  const float p2 = __fmul_rn(p, p);
+  const float p4 = __fmul_rn(p2, p2);
+  const float p8 = __fmul_rn(p4, p4);
+  const float p16 = __fmul_rn(p8, p8);
+  float r = __uint_as_float(0x7EF00000u - __float_as_uint(p16));
+#pragma unroll
+  for (int it = 0; it < 3; ++it) r = __fmul_rn(r, __fsub_rn(2.0f, __fmul_rn(p16, r)));
+  const float e = __fsub_rn(1.0f, r);
+  const float erf_u = u < 0.0f ? -e : e;
+  return __fmul_rn(__fmul_rn(0.5f, v), __fadd_rn(1.0f, erf_u));
+}
 
 // Pair tile: 256 weight rows (128 per CTA of the cluster pair) x BN rows of X
 // (BN/2 loaded by each CTA).  STAGES is the deepest operand ring that fits.
@@ -60,7 +99,7 @@ struct Cfg {
   static constexpr int MSTG_BYTES = kInt8 ? 4096 : 2048;  // canonical metadata of the stage (TMA)
   static constexpr int MCP_BYTES = kInt8 ? 0 : 2048;      // fp16/bf16: metadata in tcgen05.cp order
   static constexpr int MCOLS = kInt8 ? 8 : 4;          // TMEM columns of metadata per stage
-  static constexpr int OUT_ES = OUT == OUT_S32 ? 4 : 2;
+  static constexpr int OUT_ES = OUT == OUT_S32 ? 4 : out_s8(OUT) ? 1 : 2;
   static constexpr bool YT = OUT == OUT_F16_T || OUT == OUT_BF16_T;  // Y^T: stored from registers
   static constexpr bool OUT_BF = out_bf16(OUT);
   // staging per epilogue warp: 16-bit outputs double-buffer a 4 KB box per warp
@@ -233,7 +272,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     spgemm24_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
                     void* __restrict__ Yp, int64_t ldy, const void* __restrict__ bias,
-                    const float* __restrict__ scale, int M, int N, int K, uint32_t* err) {
+                    const float* __restrict__ scale, float qscale, int M, int N, int K, uint32_t* err) {
   using C = Cfg<kInt8, BN, OUT>;
   constexpr int STAGES = C::STAGES;
   constexpr int BNH = C::BNH;
@@ -473,6 +512,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         }
         const int mb = m0 + 32 * c;
         if (nb >= N || mb >= M) continue;
+        if constexpr (C::OUT_ES == 1) {
+          // int8 out: v = fp32(acc) *rn scale (+rn bias) [GELU], q = clamp(rne(v *rn qscale)),
+          // staged as [32 rows m][32 bytes n] in this warp's buffer; lane r stores row r
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            float v = __fmul_rn(__int2float_rn(static_cast<int>(h[k])), sc);
+            if (has_bias) v = __fadd_rn(v, badd);
+            if constexpr (out_gelu(OUT)) v = gelu_as_f32(v);
+            const int qv = max(-127, min(127, __float2int_rn(__fmul_rn(v, qscale))));
+            buf[k * 32 + lane] = static_cast<uint8_t>(qv & 0xFF);
+          }
+          __syncwarp();
+          const int row = mb + lane;
+          if (row < M) {
+            uint8_t* yrow = static_cast<uint8_t*>(Yp) + int64_t(row) * ldy + nb;
+            const uint8_t* srow = buf + lane * 32;
+            if (full_n) {
+              reinterpret_cast<uint4*>(yrow)[0] = reinterpret_cast<const uint4*>(srow)[0];
+              reinterpret_cast<uint4*>(yrow)[1] = reinterpret_cast<const uint4*>(srow)[1];
+            } else {
+              for (int e = 0; e < N - nb; ++e) yrow[e] = srow[e];
+            }
+          }
+          __syncwarp();
+          continue;
+        }
         if constexpr (C::OUT_ES == 4) {
 #pragma unroll
           for (int k = 0; k < 32; ++k) h[k] = convert_out<OUT, kInt8>(h[k], badd, sc, has_bias);
@@ -621,17 +686,26 @@ int resident_pairs(const void* kern, int smem, int threads) {
 
 template <bool kInt8, bool kBF16, int BN, int OUT>
 spg_status launch(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,
-                  const float* scale, void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t stream) {
+                  const float* scale, void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t stream,
+                  float qscale) {
   using C = Cfg<kInt8, BN, OUT>;
   const int es = kInt8 ? 1 : 2;
   CUtensorMap tmA, tmB, tmE, tmY;
   if (!make_tmap_2d(&tmA, Wv, es, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2) * es, 128 / es, 128, true) ||
       !make_tmap_2d(&tmB, X, es, uint64_t(K), uint64_t(M), uint64_t(ldx) * es, 128 / es, C::BNH, true) ||
-      !make_tmap_2d(&tmE, meta, 1, uint64_t(K / 8), uint64_t(N), uint64_t(K / 8), 16, 128, false) ||
-      !(C::YT ? make_tmap_2d_swz(&tmY, Y, 2, uint64_t(M), uint64_t(N), uint64_t(ldy) * 2, 32, 32, 64)
-              : make_tmap_2d(&tmY, Y, C::OUT_ES, uint64_t(N), uint64_t(M), uint64_t(ldy) * C::OUT_ES,
-                             C::OUT_ES == 2 ? 64 : 32, 32, C::OUT_ES == 2)))
+      !make_tmap_2d(&tmE, meta, 1, uint64_t(K / 8), uint64_t(N), uint64_t(K / 8), 16, 128, false))
     return SPG_ERR_CUDA;
+  // the output map: Y^T boxes [32 n][32 m] with 64-byte swizzle, Y boxes of 64
+  // (16-bit) or 32 (32-bit) columns x 32 rows; int8 outputs are stored without TMA
+  bool ymap_ok = true;
+  if constexpr (C::OUT_ES == 1)
+    std::memset(&tmY, 0, sizeof(tmY));
+  else if constexpr (C::YT)
+    ymap_ok = make_tmap_2d_swz(&tmY, Y, 2, uint64_t(M), uint64_t(N), uint64_t(ldy) * 2, 32, 32, 64);
+  else
+    ymap_ok = make_tmap_2d(&tmY, Y, C::OUT_ES, uint64_t(N), uint64_t(M), uint64_t(ldy) * C::OUT_ES,
+                           C::OUT_ES == 2 ? 64 : 32, 32, C::OUT_ES == 2);
+  if (!ymap_ok) return SPG_ERR_CUDA;
   uint32_t* err = device_error_word();
   if (!err) return SPG_ERR_CUDA;
   auto kern = spgemm24_kernel<kInt8, kBF16, BN, OUT>;
@@ -641,8 +715,8 @@ spg_status launch(const void* X, int64_t ldx, const void* Wv, const uint8_t* met
   const int64_t pairs_max = resident_pairs(reinterpret_cast<const void*>(kern), C::SMEM, C::THREADS);
   if (pairs_max <= 0) return SPG_ERR_CUDA;
   const int pairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
-  if (launch_pdl(kern, dim3(2 * pairs), dim3(C::THREADS), C::SMEM, stream, tmA, tmB, tmE, tmY, Y, ldy, bias, scale, static_cast<int>(M),
-                                            static_cast<int>(N), static_cast<int>(K), err) != cudaSuccess)
+  if (launch_pdl(kern, dim3(2 * pairs), dim3(C::THREADS), C::SMEM, stream, tmA, tmB, tmE, tmY, Y, ldy, bias, scale,
+                 qscale, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), err) != cudaSuccess)
     return SPG_ERR_CUDA;
   return launch_status();
 }
@@ -651,10 +725,11 @@ spg_status launch(const void* X, int64_t ldx, const void* Wv, const uint8_t* met
 // tile whose two accumulators and metadata ring fit in tensor memory.
 template <bool kInt8, bool kBF16, int OUT>
 spg_status dispatch(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,
-                    const float* scale, void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t s) {
-  if (M <= 32) return launch<kInt8, kBF16, 32, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s);
-  if (M <= 128) return launch<kInt8, kBF16, 128, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s);
-  return launch<kInt8, kBF16, 224, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s);
+                    const float* scale, void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t s,
+                    float qscale = 0.f) {
+  if (M <= 32) return launch<kInt8, kBF16, 32, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s, qscale);
+  if (M <= 128) return launch<kInt8, kBF16, 128, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s, qscale);
+  return launch<kInt8, kBF16, 224, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s, qscale);
 }
 
 spg_status validate_common(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, void* Y, int64_t ldy,
@@ -742,6 +817,27 @@ spg_status spgemm_24_s8(const int8_t* X, int64_t ldx, const int8_t* Wv, const ui
   if (out_mode == SPG_OUT_S32)
     return dispatch<true, false, OUT_S32>(X, ldx, Wv, meta, nullptr, nullptr, Y, ldy, M, N, K, s);
   return dispatch<true, false, OUT_F16>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s);
+}
+
+// int8 2:4 layer whose epilogue quantises its output for the next int8 layer
+// (optionally through GELU): the fixed-point path of the compressed ViT MLP.
+spg_status spgemm_24_s8_q(const int8_t* X, int64_t ldx, const int8_t* Wv, const uint8_t* meta, const float* scale,
+                          const void* bias, float qscale, int act, int8_t* Yq, int64_t ldy, int64_t M, int64_t N,
+                          int64_t K, spg_stream_t stream) {
+  using namespace spg;
+  using namespace spg::gemm24;
+  if (act != SPG_ACT_NONE && act != SPG_ACT_GELU) return SPG_ERR_INVALID_ARG;
+  if (!scale || !(qscale > 0.f) || !(qscale < 3.0e38f)) return SPG_ERR_INVALID_ARG;
+  spg_status st = validate_common(X, ldx, Wv, meta, Yq, ldy, M, N, K, 1, 1, 256);
+  if (st != SPG_OK) return st;
+  if (!aligned(scale, 4)) return SPG_ERR_MISALIGNED;
+  if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;
+  st = check_device();
+  if (st != SPG_OK) return st;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  if (act == SPG_ACT_GELU)
+    return dispatch<true, false, OUT_S8QG>(X, ldx, Wv, meta, bias, scale, Yq, ldy, M, N, K, s, qscale);
+  return dispatch<true, false, OUT_S8Q>(X, ldx, Wv, meta, bias, scale, Yq, ldy, M, N, K, s, qscale);
 }
 
 }  // extern "C"

@@ -196,3 +196,48 @@ def test_gelu_textbook_values_and_symmetry():
     assert s24.gelu_ref(np.array([0.0]))[0] == 0.0
     assert abs(s24.gelu_ref(np.array([10.0]))[0] - 10.0) < 1e-12
     assert abs(s24.gelu_ref(np.array([-10.0]))[0]) < 1e-12
+
+
+def test_erf_as_within_published_bound():
+    """A&S 7.1.28 in fp32 stays within its 3e-7 bound of the true erf (plus
+    fp32 rounding) -- checked against the C library's erf."""
+    import math
+    import numpy as np
+    from oracle import sparse24 as s24
+    x = np.linspace(-6, 6, 24001).astype(np.float32)
+    got = s24.erf_as_f32(x).astype(np.float64)
+    want = np.array([math.erf(float(v)) for v in x])
+    # 3e-7 for the approximation; in fp32, p carries about 2 roundings (2^-24
+    # each, relative) which the 16th power multiplies by 16, the four squarings
+    # add 4 more (36 * 2^-24 on 1/p^16), and the Newton reciprocal ends within
+    # 1.6e-7 of 1/p^16
+    assert np.max(np.abs(got - want)) <= 3e-7 + 36 * 2.0 ** -24 + 1.6e-7
+    assert s24.erf_as_f32(np.array([0.0], np.float32))[0] == 0.0
+    assert s24.erf_as_f32(np.array([40.0], np.float32))[0] == 1.0       # p^16 overflows: 1 - 1/inf
+
+
+def test_gelu_as_against_fp64_gelu_and_quantiser_rounding():
+    import numpy as np
+    from oracle import sparse24 as s24
+    v = np.linspace(-12, 40, 52001).astype(np.float32)
+    got = s24.gelu_as_f32(v).astype(np.float64)
+    want = s24.gelu_ref(v.astype(np.float64))
+    # |GELU error| <= 0.5 |v| |erf error| plus three fp32 roundings of the result
+    bound = 0.5 * np.abs(v) * (3e-7 + 36 * 2.0 ** -24 + 1.6e-7) + 3 * 2.0 ** -24 * np.maximum(1.0, np.abs(want))
+    assert np.all(np.abs(got - want) <= bound)
+    # the quantiser: round half to even, clamp to +-127; scale 0.5 and qscale 1 make v = acc / 2
+    acc = np.array([[5, 7, -5, 1000, -1000, 3, 0]], dtype=np.int64)
+    q = s24.quantize_s8(acc, np.full(7, 0.5, np.float32), None, 1.0, False)
+    assert q.tolist() == [[2, 4, -2, 127, -127, 2, 0]]
+    # GELU before the quantiser: GELU(-x) is small and negative, GELU(large) = x
+    q = s24.quantize_s8(np.array([[-2, 40]]), np.ones(2, np.float32), None, 100.0, True)
+    assert q.tolist() == [[-5, 127]]          # GELU(-2) = -0.0455 -> -4.55 -> -5
+
+
+def test_erf_as_is_exactly_one_from_four():
+    """The definition clamps |u| at 4, where the fp32 value is already 1.0."""
+    import numpy as np
+    from oracle import sparse24 as s24
+    assert s24.erf_as_f32(np.array([4.0], np.float32))[0] == 1.0
+    x = np.concatenate([np.linspace(4, 80, 200001), np.geomspace(80, 3e38, 20001)]).astype(np.float32)
+    assert (s24.erf_as_f32(x) == 1.0).all() and (s24.erf_as_f32(-x) == -1.0).all()

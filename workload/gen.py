@@ -151,6 +151,9 @@ CONFIGS: Dict[str, Config] = {
     "vitl_mlp_s8": Config(
         "vitl_mlp_s8", "24_s8", (("fc1", 6304, 4096, 1024, False),),
         note="2:4 int8 ViT-Large MLP fc1, M=32x197, per-row symmetric int8 weights"),
+    "vitl_mlp_chain_s8": Config(
+        "vitl_mlp_chain_s8", "24_s8", (("fc1", 6304, 4096, 1024, True), ("fc2", 6304, 1024, 4096, True)),
+        note="2:4 int8 ViT-Large MLP block: fc1 (+bias, GELU, int8 quantisation) -> fc2 (+bias) -> fp16"),
     "tw_bert_f16": Config(
         "tw_bert_f16", "tw_f16",
         (("attn_out", 4096, 768, 768, False), ("ffn_in", 4096, 3072, 768, False)),
@@ -187,7 +190,19 @@ def _layer_inputs(cfg: Config, seed: int, lname: str, M: int, N: int, K: int, bi
         q = np.clip(np.rint(w / s[:, None]), -127, 127).astype(np.int8)
         d["W"] = q
         d["scale"] = s
-        d["bias"] = None
+        d["bias"] = f32_to_f16(normal(seed, stem + ".bias", N, cfg.bias_std)) if bias else None
+        if cfg.name == "vitl_mlp_chain_s8":
+            # Static activation scale of fc1's output (fc2's int8 input): 4 standard
+            # deviations of the dequantised fc1 value map to 127.  The deviation
+            # follows from the stated distributions: int8 X uniform on [-127, 127]
+            # (std sqrt((255^2 - 1) / 12)), weights N(0, w_std), K/2 kept products.
+            sigma = np.sqrt((255.0 ** 2 - 1.0) / 12.0) * cfg.w_std * np.sqrt(1024 / 2.0)
+            act_scale = np.float32(4.0 * sigma / 127.0)
+            if lname == "fc1":
+                d["qscale"] = np.float32(1.0) / act_scale      # fc1's epilogue quantises with this
+            else:
+                d["X"] = None                                  # fc2's input is fc1's int8 output
+                d["scale"] = (s * act_scale).astype(np.float32)  # activation scale folded in
         return d
     to = f32_to_bf16_bits if cfg.kind == "24_bf16" else f32_to_f16
     d["X"] = to(normal(seed, stem + ".X", M * K, cfg.x_std)).reshape(M, K)
