@@ -33,7 +33,9 @@ from workload import gen  # noqa: E402
 METRIC = "sparse GEMM dense-equiv TFLOP/s and % of B200 sparse tensor peak (or HBM GB/s)"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
-DTYPE_NAME = {"24_f16": "f16", "24_bf16": "bf16", "24_s8": "s8", "tw_f16": "f16"}
+# fp32 pipe peak of the CUDA-core tile-wise path: SM count, fp32 lanes per SM, maximum SM clock
+FP32_SMS, FP32_LANES, FP32_MAX_MHZ = 148, 128, 1965
+DTYPE_NAME = {"24_f16": "f16", "24_bf16": "bf16", "24_s8": "s8", "tw_f16": "f16", "tw_f32": "f32"}
 
 
 def load_peaks():
@@ -236,7 +238,33 @@ class LayerTW:
             self.spg.spgemm_tw_f16(X, self.desc, self.x_layout, Y=Y, workspace=self.ws, M=self.d["M"])
 
 
-def tw_algorithmic(layers_tw):
+class LayerTW32:
+    """fp32 tile-wise layer on the CUDA cores: the pattern selected on the fp16
+    copy of W, the fp32 weights condensed through it."""
+
+    def __init__(self, spg, d, copies, x_layout):
+        import torch
+        self.spg, self.d, self.y_nm = spg, d, False
+        dev = torch.device("cuda")
+        self.desc = spg.tw_reorganize(torch.from_numpy(d["W16"]).to(dev), d["G"], d["n_pruned"],
+                                      list(d["k_per_tile"]))
+        self.Wc32 = spg.tw_condense_f32(torch.from_numpy(d["W"]).to(dev), self.desc)
+        X = torch.from_numpy(d["X"]).to(dev)
+        if x_layout == spg.SPG_X_KM:
+            X = X.t().contiguous()
+        self.x_layout = x_layout
+        self.X = [X] + [X.clone() for _ in range(copies - 1)]
+        self.Y = [torch.empty((d["M"], d["N"]), dtype=torch.float32, device=dev) for _ in range(copies)]
+        ws = int(spg.lib().tw_workspace_size_f32(d["M"], d["K"], x_layout))
+        self.ws = torch.empty(max(ws, 256), dtype=torch.uint8, device=dev)
+
+    def run(self, i, X=None, Y=None):
+        X = self.X[i] if X is None else X
+        Y = self.Y[i] if Y is None else Y
+        self.spg.spgemm_tw_f32(X, self.desc, self.Wc32, self.x_layout, Y=Y, workspace=self.ws, M=self.d["M"])
+
+
+def tw_algorithmic(layers_tw, es=2):
     flops = 0.0
     byts = 0
     for L in layers_tw:
@@ -246,7 +274,7 @@ def tw_algorithmic(layers_tw):
         G = d["G"]
         gts = [min(G, Nk - t * G) for t in range(len(kp))]
         flops += 2.0 * d["M"] * sum(g * k for g, k in zip(gts, kp))
-        byts += 2 * d["M"] * d["K"] + 2 * d["M"] * d["N"] + 2 * sum(g * k for g, k in zip(gts, kp))
+        byts += es * (d["M"] * d["K"] + d["M"] * d["N"] + sum(g * k for g, k in zip(gts, kp)))
     return flops, byts
 
 
@@ -259,14 +287,20 @@ def run_ours(args, rank, world, local_rank):
     inputs = gen.make_inputs(args.workload)
     kind = cfg.kind
     # rotating buffer sets: enough that the sets one step cycles through exceed 3x the 126 MB L2
-    if kind == "tw_f16":
-        step_bytes = sum(2 * d["M"] * d["K"] * (2 if not args.x_km else 1) + 2 * d["M"] * d["N"] for d in inputs)
+    if kind in ("tw_f16", "tw_f32"):
+        es = 4 if kind == "tw_f32" else 2
+        step_bytes = sum(es * (d["M"] * d["K"] * (2 if not args.x_km else 1) + d["M"] * d["N"]) for d in inputs)
     else:
         step_bytes = sum(algorithmic_bytes(d, kind) for d in inputs)
     copies = max(args.copies, int(math.ceil(3 * L2_BYTES / step_bytes)))
     if kind == "tw_f16":
         layers = [LayerTW(spg, d, copies, spg.SPG_X_KM if args.x_km else spg.SPG_X_MK, args.y_nm) for d in inputs]
         flops_alg, bytes_alg = tw_algorithmic(layers)
+    elif kind == "tw_f32":
+        if args.y_nm:
+            raise SystemExit("--y-nm applies to the fp16 tile-wise and 2:4 workloads")
+        layers = [LayerTW32(spg, d, copies, spg.SPG_X_KM if args.x_km else spg.SPG_X_MK) for d in inputs]
+        flops_alg, bytes_alg = tw_algorithmic(layers, es=4)
     else:
         if args.y_nm and kind not in ("24_f16", "24_bf16"):
             raise SystemExit("--y-nm applies to the 16-bit 2:4 and tile-wise workloads")
@@ -365,14 +399,24 @@ def run_ours(args, rank, world, local_rank):
 
     peaks, src = load_peaks()
     lay_ms = [float(np.mean(p)) for p in per_layer]
-    if kind == "24_bf16" and inputs[0]["M"] <= 64 or kind == "tw_f16":
+    if kind == "tw_f32":
+        # fp32 fused multiply-add on the CUDA cores: kept FLOPs per launch against the fp32 pipe
+        # peak, 148 SMs x 128 lanes x 2 FLOPs at the 1965 MHz maximum SM clock
+        peak = FP32_SMS * FP32_LANES * 2 * FP32_MAX_MHZ * 1e6 / 1e12
+        achieved = flops_alg / nl / (np.mean(lay_ms) * 1e-3) / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
+                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
+                "scope": "whole library call per layer" + ("" if args.x_km else " (includes the [M, K] -> [K, M] transpose)"),
+                "kernel": "tw_gemm_f32_kernel"}
+    elif kind == "24_bf16" and inputs[0]["M"] <= 64 or kind == "tw_f16":
         # HBM-bound shapes: algorithmic bytes per launch over the measured copy bandwidth
         per_launch_bytes = bytes_alg / nl
         achieved = per_launch_bytes / (np.mean(lay_ms) * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic(args.workload),
                 "peak_source": src,
-                "kernel": "spgemm24_kernel" if kind != "tw_f16" else "tw_gemm_kernel"}
+                "kernel": "tw_gemm_kernel" if kind == "tw_f16" else "spgemm24_kernel"}
     else:
         # dense-equivalent FLOPs per launch against the 2:4 sparse tensor peak of the dtype:
         # measured dense bf16 (same rate as fp16) x2 for 2:4 sparsity, x2 again for int8
@@ -399,7 +443,7 @@ def run_ours(args, rank, world, local_rank):
         "per_layer_us": [1e3 * v for v in lay_ms],
         "roofline": roof,
         "e2e": e2e,
-        "gpu_launches": args.steps * nl * (2 if (kind == "tw_f16" and not args.x_km) else 1),
+        "gpu_launches": args.steps * nl * (2 if (kind in ("tw_f16", "tw_f32") and not args.x_km) else 1),
         "dense_cublas": dense,
         "clocks": clocks,
     }
@@ -424,14 +468,14 @@ def dense_baseline(layers, kind, copies, reps, gstream, stream, args):
             fn = lambda i, L=L, Wd=Wd: torch._int_mm(L.X[i], Wd[i])
         else:
             tdt = L.X[0].dtype
-            if kind == "tw_f16":
+            if kind in ("tw_f16", "tw_f32"):
                 W = torch.from_numpy(np.ascontiguousarray(d["W"])).to(dev)
             else:
                 W = Layer24._t(d["W"], tdt, dev)
             Wd = [W.t()] + [W.clone().t() for _ in range(copies - 1)]
             bias = getattr(L, "bias", [None])[0]
             use_gelu = getattr(L, "gelu", False)
-            xs = L.X if not (kind == "tw_f16" and L.x_layout == 1) else [x.t() for x in L.X]
+            xs = L.X if not (kind in ("tw_f16", "tw_f32") and L.x_layout == 1) else [x.t() for x in L.X]
 
             def fn(i, xs=xs, Wd=Wd, bias=bias, use_gelu=use_gelu):
                 # nn.functional.linear: one cuBLAS(Lt) GEMM with the bias in its epilogue
@@ -509,6 +553,9 @@ def oracle_step(inputs, kind, rows_frac=1.0):
             M = len(rows)
         if kind == "tw_f16":
             r = tw.tw_reorganize(d["W"], d["G"], d["n_pruned"], d["k_per_tile"])
+            tw.tw_gemm_ref(d["X"], r, rows=rows)
+        elif kind == "tw_f32":
+            r = tw.tw_condense_values(d["W"], tw.tw_reorganize(d["W16"], d["G"], d["n_pruned"], d["k_per_tile"]))
             tw.tw_gemm_ref(d["X"], r, rows=rows)
         elif kind == "24_s8":
             Wv, meta = s24.compress_24(d["W"], "s8")

@@ -299,6 +299,30 @@ spg_status spgemm_tw_f16_yt(const void* X, int64_t ldx, int x_layout, const spg_
                             int64_t ldyt, int64_t M, void* workspace, size_t ws_bytes, spg_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Tile-wise sparsity on the CUDA cores in fp32  [TW, library table (the
+ * tile-wise CUDA-fp32 library) and results slide (speedup on CUDA cores)]
+ *
+ * The pattern of a descriptor filled by tw_reorganize (selected exactly on
+ * the fp16 copy of the weights) applied to fp32 weights and activations:
+ *   tw_condense_f32: Wc32 [tile_kofs[T]/64][G][64] fp32 (the layout of the
+ *     descriptor's Wc), Wc32[blk][j][c] = W[offsetn[tG+j]][offsetk[tile_kofs[t]
+ *     + 64b + c]] for j < G_t and 64b + c < k_t, +0 elsewhere; W fp32 [N, K],
+ *     pitch ldw >= K, 4-byte aligned; Wc32 16-byte aligned.
+ *   spgemm_tw_f32: Y [M, N] fp32 = X . Wd^T with Wd the fp32 tile-wise weight,
+ *     on the fp32 pipes (fused multiply-add, each tile's kept rows in
+ *     ascending order); pruned columns of Y are +0.  X fp32 [M, K] pitch ldx
+ *     (SPG_X_MK; first transposed into `workspace`, ws_bytes >=
+ *     tw_workspace_size_f32) or [K, M] (SPG_X_KM; 16-byte aligned, ldx a
+ *     multiple of 4).  Y 4-byte aligned, any ldy >= N.  M <= 65535 * 128.
+ * ------------------------------------------------------------------------- */
+spg_status tw_condense_f32(const float* W, int64_t ldw, const spg_tw_desc* desc, float* Wc32, spg_stream_t stream);
+
+size_t tw_workspace_size_f32(int64_t M, int64_t K, int x_layout);
+
+spg_status spgemm_tw_f32(const float* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, const float* Wc32,
+                         float* Y, int64_t ldy, int64_t M, void* workspace, size_t ws_bytes, spg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * spgemm_tw_f16_noalloc  (no counterpart on the pages: an interface addition)
  *
  * spgemm_tw_f16 with x_layout SPG_X_MK for callers that cannot allocate device

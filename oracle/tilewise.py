@@ -112,19 +112,33 @@ def tw_reorganize(W: np.ndarray, G: int, n_pruned: int, k_per_tile) -> dict:
             "col_keys": ckeys}
 
 
+def tw_condense_values(W: np.ndarray, tw: dict) -> dict:
+    """The same pattern carrying the values of another weight W [N, K] (for the
+    fp32 library: the pattern is selected on the fp16 copy, the values are the
+    fp32 weights): tile t's Wc = W[cols_t][:, offsetk_t] in W's dtype."""
+    W = np.asarray(W)
+    out = dict(tw)
+    out["tiles"] = [dict(t, Wc=W[np.ix_(t["cols"], t["offsetk"])].copy()) for t in tw["tiles"]]
+    return out
+
+
 def tw_expand(tw: dict) -> np.ndarray:
-    """Dense fp16 [N, K] equal to W masked by (kept column and kept row of its tile)."""
-    Wd = np.zeros((tw["N"], tw["K"]), dtype=np.float16)
+    """Dense [N, K] (the tiles' dtype) equal to W masked by (kept column and kept row of its tile)."""
+    Wd = np.zeros((tw["N"], tw["K"]), dtype=tw["tiles"][0]["Wc"].dtype)
     for tile in tw["tiles"]:
         Wd[np.ix_(tile["cols"], tile["offsetk"])] = tile["Wc"]
     return Wd
 
 
 def tw_gemm_ref(X: np.ndarray, tw: dict, rows=None) -> np.ndarray:
-    """fp64 reference Y = X . Wd^T of the tile-wise layer (pruned columns exactly 0)."""
+    """fp64 reference Y = X . Wd^T of the tile-wise layer (pruned columns exactly 0).
+    X and the tiles keep their own precision (fp16 or fp32), converted exactly."""
     Xs = X if rows is None else X[rows]
     Wd = tw_expand(tw).astype(np.float64)
-    return np.asarray(Xs, dtype=np.float16).astype(np.float64) @ Wd.T
+    Xs = np.asarray(Xs)
+    if Xs.dtype != np.float32:
+        Xs = Xs.astype(np.float16)
+    return Xs.astype(np.float64) @ Wd.T
 
 
 def achieved_sparsity(tw: dict) -> float:

@@ -62,6 +62,10 @@ SIGNATURES = {
                                      _sz, _p]),
     "spgemm_tw_f16_yt": (ctypes.c_int, [_p, _i64, ctypes.c_int, ctypes.POINTER(SpgTwDesc), _p, _i64, _i64, _p,
                                         _sz, _p]),
+    "tw_condense_f32": (ctypes.c_int, [_p, _i64, ctypes.POINTER(SpgTwDesc), _p, _p]),
+    "tw_workspace_size_f32": (_sz, [_i64, _i64, ctypes.c_int]),
+    "spgemm_tw_f32": (ctypes.c_int, [_p, _i64, ctypes.c_int, ctypes.POINTER(SpgTwDesc), _p, _p, _i64, _i64, _p, _sz,
+                                     _p]),
     "spgemm_tw_f16_noalloc": (ctypes.c_int, [_p, _i64, ctypes.POINTER(SpgTwDesc), _p, _i64, _i64, _p]),
 }
 
@@ -293,6 +297,34 @@ def spgemm_tw_f16_yt(X, desc: TwDesc, x_layout=SPG_X_MK, Yt=None, workspace=None
         _ptr(X), X.stride(0), x_layout, ctypes.byref(desc.c), _ptr(Yt), Yt.stride(0), M, _ptr(workspace),
         ws if workspace is not None else 0, _stream(stream)))
     return Yt
+
+
+def tw_condense_f32(W, desc: TwDesc, Wc32=None, stream=None):
+    """fp32 condensed tiles of W [N, K] (fp32) through the pattern of ``desc``."""
+    import torch
+    if Wc32 is None:
+        Wc32 = torch.empty(desc.sizes.wc_elems, dtype=torch.float32, device=W.device)
+    _check("tw_condense_f32", lib().tw_condense_f32(_ptr(W), W.stride(0), ctypes.byref(desc.c), _ptr(Wc32),
+                                                    _stream(stream)))
+    return Wc32
+
+
+def spgemm_tw_f32(X, desc: TwDesc, Wc32, x_layout=SPG_X_MK, Y=None, workspace=None, M: Optional[int] = None,
+                  stream=None):
+    """Tile-wise GEMM in fp32 on the CUDA cores: X [M, K] or [K, M] -> Y [M, N] fp32."""
+    import torch
+    if M is None:
+        M = X.shape[0] if x_layout == SPG_X_MK else X.shape[1]
+    N = desc.sizes.N
+    if Y is None:
+        Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
+    ws = int(lib().tw_workspace_size_f32(M, desc.sizes.K, x_layout))
+    if workspace is None and ws:
+        workspace = torch.empty(ws, dtype=torch.uint8, device=X.device)
+    _check("spgemm_tw_f32", lib().spgemm_tw_f32(
+        _ptr(X), X.stride(0), x_layout, ctypes.byref(desc.c), _ptr(Wc32), _ptr(Y), Y.stride(0), M, _ptr(workspace),
+        ws if workspace is not None else 0, _stream(stream)))
+    return Y
 
 
 def spgemm_tw_f16_noalloc(X, desc: TwDesc, Y=None, stream=None):

@@ -126,3 +126,27 @@ def test_bert_shapes_counts_and_sparsity():
         assert len(r["offsetn"]) == Nk and r["T"] == T
         assert [len(t["cols"]) for t in r["tiles"]][-1] == Nk - (T - 1) * 128
         assert abs(tw.achieved_sparsity(r) - 0.75) <= 0.05
+
+
+def test_fp32_values_through_the_fp16_pattern():
+    """The fp32 library: the pattern selected on the fp16 copy carries the fp32
+    values; its reference equals a triple loop over (kept column, kept row)."""
+    import numpy as np
+    from oracle import tilewise as tw
+    rng = np.random.default_rng(4)
+    N, K, M, P = 40, 64, 5, 6
+    W32 = (rng.standard_normal((N, K)) * 0.3).astype(np.float32)
+    X32 = rng.standard_normal((M, K)).astype(np.float32)
+    kpt = [17]
+    r16 = tw.tw_reorganize(W32.astype(np.float16), 128, P, kpt)
+    r32 = tw.tw_condense_values(W32, r16)
+    assert r32["tiles"][0]["Wc"].dtype == np.float32
+    Y = tw.tw_gemm_ref(X32, r32)
+    want = np.zeros((M, N))
+    for t in r32["tiles"]:
+        for jj, n in enumerate(t["cols"]):
+            for ii, k in enumerate(t["offsetk"]):
+                assert t["Wc"][jj, ii] == W32[n, k]
+                want[:, n] += X32[:, k].astype(np.float64) * float(W32[n, k])
+    assert np.array_equal(Y, want) or np.allclose(Y, want, rtol=1e-15, atol=1e-15)
+    assert set(np.nonzero(np.abs(Y).sum(axis=0))[0]) <= set(r32["offsetn"])

@@ -122,7 +122,7 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
 class Config:
     """One synthetic workload.
 
-    kind: "24_f16" | "24_bf16" | "24_s8" | "tw_f16".
+    kind: "24_f16" | "24_bf16" | "24_s8" | "tw_f16" | "tw_f32".
     layers: list of (name, M, N, K, bias) GEMMs making up one pass.
     """
 
@@ -159,6 +159,11 @@ CONFIGS: Dict[str, Config] = {
         (("attn_out", 4096, 768, 768, False), ("ffn_in", 4096, 3072, 768, False)),
         G=128, col_prune_frac=0.10, density_lo=0.15, density_hi=0.40,
         note="tile-wise fp16 BERT-base shapes, M=32x128, G=128, ~75% sparse"),
+    "tw_bert_f32": Config(
+        "tw_bert_f32", "tw_f32",
+        (("attn_out", 4096, 768, 768, False), ("ffn_in", 4096, 3072, 768, False)),
+        G=128, col_prune_frac=0.10, density_lo=0.15, density_hi=0.40,
+        note="tile-wise fp32 (CUDA cores) BERT-base shapes, M=32x128, G=128, ~75% sparse"),
     "bf16_prefill": Config(
         "bf16_prefill", "24_bf16", (("proj", 8192, 16384, 4096, False),),
         shared_w="bf16_large",
@@ -205,10 +210,14 @@ def _layer_inputs(cfg: Config, seed: int, lname: str, M: int, N: int, K: int, bi
                 d["scale"] = (s * act_scale).astype(np.float32)  # activation scale folded in
         return d
     to = f32_to_bf16_bits if cfg.kind == "24_bf16" else f32_to_f16
+    if cfg.kind == "tw_f32":   # fp32 data; the pattern is selected on the fp16 copy W16
+        to = lambda a: np.asarray(a, dtype=np.float32)
     d["X"] = to(normal(seed, stem + ".X", M * K, cfg.x_std)).reshape(M, K)
     d["W"] = to(normal(seed, wstem + ".W", N * K, cfg.w_std)).reshape(N, K)
+    if cfg.kind == "tw_f32":
+        d["W16"] = f32_to_f16(d["W"])
     d["bias"] = to(normal(seed, stem + ".bias", N, cfg.bias_std)) if bias else None
-    if cfg.kind == "tw_f16":
+    if cfg.kind in ("tw_f16", "tw_f32"):
         P, Nk, T = tw_tile_counts(N, cfg.G, cfg.col_prune_frac)
         u = uniform01(seed, stem + ".density", T)
         dens = cfg.density_lo + (cfg.density_hi - cfg.density_lo) * u
