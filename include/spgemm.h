@@ -304,16 +304,19 @@ spg_status spgemm_tw_f16_yt(const void* X, int64_t ldx, int x_layout, const spg_
  *
  * The pattern of a descriptor filled by tw_reorganize (selected exactly on
  * the fp16 copy of the weights) applied to fp32 weights and activations:
- *   tw_condense_f32: Wc32 [tile_kofs[T]/64][G][64] fp32 (the layout of the
- *     descriptor's Wc), Wc32[blk][j][c] = W[offsetn[tG+j]][offsetk[tile_kofs[t]
- *     + 64b + c]] for j < G_t and 64b + c < k_t, +0 elsewhere; W fp32 [N, K],
- *     pitch ldw >= K, 4-byte aligned; Wc32 16-byte aligned.
+ *   tw_condense_f32: Wc32 [tile_kofs[T]/64][64][G] fp32, k-major (the
+ *     descriptor's Wc has the same elements with j and c swapped): block b of
+ *     tile t at blk = tile_kofs[t]/64 + b holds Wc32[blk][c][j] =
+ *     W[offsetn[tG+j]][offsetk[tile_kofs[t] + 64b + c]] for j < G_t and
+ *     64b + c < k_t, +0 elsewhere; W fp32 [N, K], pitch ldw >= K, 4-byte
+ *     aligned; Wc32 16-byte aligned, as many elements as the descriptor's Wc.
  *   spgemm_tw_f32: Y [M, N] fp32 = X . Wd^T with Wd the fp32 tile-wise weight,
  *     on the fp32 pipes (fused multiply-add, each tile's kept rows in
  *     ascending order); pruned columns of Y are +0.  X fp32 [M, K] pitch ldx
- *     (SPG_X_MK; first transposed into `workspace`, ws_bytes >=
- *     tw_workspace_size_f32) or [K, M] (SPG_X_KM; 16-byte aligned, ldx a
- *     multiple of 4).  Y 4-byte aligned, any ldy >= N.  M <= 65535 * 128.
+ *     (SPG_X_MK; first transposed into `workspace`, 16-byte aligned,
+ *     ws_bytes >= tw_workspace_size_f32) or [K, M] (SPG_X_KM; 16-byte
+ *     aligned, ldx a multiple of 4).  Y 4-byte aligned, any ldy >= N.
+ *     M < 2^31 and T * ceil(M / 64) < 2^31 (else SPG_ERR_UNSUPPORTED_SHAPE).
  * ------------------------------------------------------------------------- */
 spg_status tw_condense_f32(const float* W, int64_t ldw, const spg_tw_desc* desc, float* Wc32, spg_stream_t stream);
 
