@@ -50,6 +50,7 @@ def load_peaks():
 PROFILED = {  # workload -> (profile summary, kernel sources whose hash it records)
     "vitb_mlp_f16": ("spgemm24_kernel.vitb_mlp_f16.md", ["spgemm24.cu", "sm100.cuh"]),
     "tw_bert_f16": ("tw_gemm_kernel.tw_bert_f16.md", ["tw.cu", "sm100.cuh"]),
+    "tw_bert_f32": ("tw_gemm_f32_kernel.tw_bert_f32.md", ["tw32.cu", "host.cuh"]),
 }
 
 
@@ -499,8 +500,10 @@ def dense_baseline(layers, kind, copies, reps, gstream, stream, args):
         torch.cuda.synchronize()
         per_layer.append(a.elapsed_time(b) / (reps * copies) * 1e3)
         del g, outs, Wd
-    return {"per_layer_us": per_layer,
-            "what": "torch.nn.functional.linear (+ gelu) / torch._int_mm (cuBLAS), dense weights of the same shapes"}
+    what = "torch.nn.functional.linear (+ gelu) / torch._int_mm (cuBLAS), dense weights of the same shapes"
+    if kind == "tw_f32":
+        what += f"; fp32 with torch.backends.cuda.matmul.allow_tf32={torch.backends.cuda.matmul.allow_tf32}"
+    return {"per_layer_us": per_layer, "what": what}
 
 
 def measure_e2e(spg, layers, kind, args, stream):
