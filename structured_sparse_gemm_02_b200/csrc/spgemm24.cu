@@ -400,7 +400,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     if (leader && lane == 0) {
       constexpr uint32_t kFmt = kInt8 ? 1u : (kBF16 ? 1u : 0u);
       constexpr uint32_t kCFmt = kInt8 ? 2u : 1u;
+      // Shared-memory descriptors of stage 0.  The start address sits in the
+      // low 14 bits as address / 16 and every operand stays below 256 KB, so
+      // the descriptor of a stage (and of a K step inside it) is the stage-0
+      // descriptor plus its byte offset / 16: nothing is rebuilt per stage.
+      const uint64_t a_desc0 = smem_desc(smem_addr(smem + C::OFF_A), 16, 1024, LAYOUT_SW128);
+      const uint64_t b_desc0 = smem_desc(smem_addr(smem + C::OFF_B), 16, 1024, LAYOUT_SW128);
+      const uint64_t e_desc0 =
+          smem_desc(smem_addr(smem + (kInt8 ? C::OFF_MSTG : C::OFF_MCP)), 2048, 128, LAYOUT_NONE);
+      constexpr uint64_t kAStep = C::A_BYTES >> 4, kBStep = C::B_BYTES >> 4;
+      constexpr uint64_t kEStep = (kInt8 ? C::MSTG_BYTES : C::MCP_BYTES) >> 4;
       uint32_t g = 0;
+      int s = 0;
+      uint32_t ph = 0;
       int i = 0;
       bool ok = true;
       for (int t = pair; ok && t < total; t += npairs, ++i) {
@@ -409,8 +421,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         tc_fence_after();
         const uint32_t acc = tmem + uint32_t(b * BN);
         for (int kb = 0; kb < KB; ++kb, ++g) {
-          const int s = g % STAGES;
-          const uint32_t ph = (g / STAGES) & 1;
           if (!mbar_wait(&full[s], ph, abort_flag, err, ERR_WAIT_FULL)) {
             ok = false;
             break;
@@ -422,27 +432,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
             }
           }
           tc_fence_after();
-          const uint32_t a_s = smem_addr(smem + C::OFF_A + s * C::A_BYTES);
-          const uint32_t b_s = smem_addr(smem + C::OFF_B + s * C::B_BYTES);
+          const uint64_t ad = a_desc0 + uint64_t(s) * kAStep;
+          const uint64_t bd = b_desc0 + uint64_t(s) * kBStep;
+          const uint64_t ed = e_desc0 + uint64_t(s) * kEStep;
           const uint32_t ecol = tmem + C::META_COL + (g & 1) * C::MCOLS;
-          if constexpr (kInt8) {
-            const uint32_t e_s = smem_addr(smem + C::OFF_MSTG + s * C::MSTG_BYTES);
-            tc_cp_128x128b_pair(ecol, smem_desc(e_s, 2048, 128, LAYOUT_NONE));
-            tc_cp_128x128b_pair(ecol + 4, smem_desc(e_s + 2048, 2048, 128, LAYOUT_NONE));
-          } else {
-            const uint32_t e_s = smem_addr(smem + C::OFF_MCP + s * C::MCP_BYTES);
-            tc_cp_128x128b_pair(ecol, smem_desc(e_s, 2048, 128, LAYOUT_NONE));
-          }
+          tc_cp_128x128b_pair(ecol, ed);
+          if constexpr (kInt8) tc_cp_128x128b_pair(ecol + 4, ed + (2048 >> 4));
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint64_t adesc = smem_desc(a_s + 32 * j, 16, 1024, LAYOUT_SW128);
-            const uint64_t bdesc = smem_desc(b_s + (j >> 1) * (BNH * 128) + (j & 1) * 64, 16, 1024, LAYOUT_SW128);
+            const uint64_t adesc = ad + uint64_t((32 * j) >> 4);
+            const uint64_t bdesc = bd + uint64_t(((j >> 1) * (BNH * 128) + (j & 1) * 64) >> 4);
             const uint32_t e = kInt8 ? ecol + 2 * j : ecol + (j & ~1);
             const uint32_t sel = kInt8 ? 0u : uint32_t(j & 1);
             tc_mma_sp_pair<kInt8>(acc, adesc, bdesc, e, instr_desc(kFmt, kCFmt, 256, BN, true, sel),
                                   (kb | j) != 0 ? 1u : 0u);
           }
           tc_commit_pair(&empty[s], 0x3);
+          if (++s == STAGES) {
+            s = 0;
+            ph ^= 1u;
+          }
         }
         if (!ok) break;
         tc_commit_pair(&acc_full[b], 0x3);
