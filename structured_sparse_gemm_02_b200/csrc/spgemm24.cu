@@ -8,18 +8,23 @@
 // rows m), and the fp32/s32 accumulator D[n][m] lives in tensor memory
 // (lane = n, column = m).  A tile of Y^T is 128 x BN.
 //
-// Persistent kernel, one CTA per SM, warp roles (256 threads):
+// Persistent kernel on cluster pairs, one CTA per SM, warp roles (384 threads):
 //   warp 0     TMA producer: compressed W, X and the canonical metadata of
 //              every stage into a STAGES-deep ring that runs across tiles
 //   warp 1     fp16/bf16 only: rearranges each stage's metadata into the
-//              order the tensor cores read it (permute_meta_f16)
+//              order the tensor cores read it (permute_meta_f16), then
+//              arrives on the leader's barrier of the stage, which completes
+//              once both CTAs' operands have landed and both metadata warps
+//              have arrived
 //   warp 2     TMEM owner and MMA issuer (one thread of the leader CTA):
-//              tcgen05.cp (metadata into tensor memory), tcgen05.mma.sp into
-//              one of two accumulators
+//              waits for a stage, then issues it (tcgen05.cp of the
+//              metadata into tensor memory, tcgen05.mma.sp into one of two
+//              accumulators) and commits the stage's slot
 //   warp 3     idle
-//   warps 4-7  epilogue: tcgen05.ld of a finished accumulator (released as
-//              soon as it is read), bias / dequant, convert, TMA store of
-//              32x32 output boxes; the ragged right edge uses checked stores
+//   warps 4-11 epilogue, two warps per tensor-memory lane quadrant:
+//              tcgen05.ld of a finished accumulator (released as soon as it
+//              is read), bias / dequant, convert, TMA store of output boxes;
+//              the ragged right edge uses checked stores
 // Every wait is bounded (sm100.cuh); on a timeout the CTA drains what it has
 // in flight, frees tensor memory and exits with the error word set.
 #include <cuda.h>
@@ -89,6 +94,13 @@ __device__ __forceinline__ float gelu_as_f32(float v) {
 
 // Pair tile: 256 weight rows (128 per CTA of the cluster pair) x BN rows of X
 // (BN/2 loaded by each CTA).  STAGES is the deepest operand ring that fits.
+// Stages waited for before their MMAs are issued.  A wait between two groups
+// of MMAs leaves the tensor pipe idle for a while, which larger groups
+// amortise, but waiting for a second stage delays the first one's MMAs while
+// the ring is short of loads; on the ViT-Base MLP shapes a group of two was
+// slower than one (42.0 / 42.6 against 40.1 / 39.2 us).
+constexpr int kIssueGroup = 1;
+
 template <bool kInt8, int BN, int OUT>
 struct Cfg {
   static constexpr int BMC = 128;                      // weight rows per CTA (MMA M = 256 per pair)
@@ -106,7 +118,7 @@ struct Cfg {
   // pair (2 KB per warp and buffer); int32 outputs one 4 KB box per warp
   static constexpr int EPI_BUF = OUT_ES == 2 ? 2 * 2048 : 4096;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + MSTG_BYTES + MCP_BYTES;
-  // full[S], mtma[S], meta_full[S], empty[S], acc_full[2], acc_empty[2], mma_done
+  // full[S], mtma[S], empty[S], acc_full[2], acc_empty[2], mma_done
   static constexpr int EPI_WARPS = 8;                  // two per tensor-memory lane quadrant
   static constexpr int THREADS = 32 * (4 + EPI_WARPS);
   static constexpr int NCH = BN / 32;                  // 32-column chunks of an accumulator
@@ -120,7 +132,7 @@ struct Cfg {
   static constexpr int OFF_MCP = OFF_MSTG + STAGES * MSTG_BYTES;
   static constexpr int OFF_EPI = OFF_MCP + STAGES * MCP_BYTES;
   static constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * EPI_BUF;
-  static constexpr int NUM_BARS = 4 * STAGES + 5;
+  static constexpr int NUM_BARS = 3 * STAGES + 5;
   static constexpr int SMEM = OFF_BAR + NUM_BARS * 8 + 16 + 1024;
   static constexpr uint32_t META_COL = 2 * BN;  // metadata ring after the two accumulators
   static constexpr uint32_t TMEM_NEED = 2 * BN + 2 * MCOLS;
@@ -280,8 +292,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* mtma = full + STAGES;
-  uint64_t* meta_full = mtma + STAGES;
-  uint64_t* empty = meta_full + STAGES;
+  uint64_t* empty = mtma + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* acc_empty = acc_full + 2;
   uint64_t* mma_done = acc_empty + 2;
@@ -298,9 +309,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      // operand bytes of both CTAs plus, for fp16/bf16, one arrival from each
+      // CTA's metadata warp once the stage's metadata is arranged
+      mbar_init(&full[s], kInt8 ? 1 : 3);
       mbar_init(&mtma[s], 1);
-      mbar_init(&meta_full[s], 2);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -330,7 +342,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   griddep_wait();  // the previous kernel's writes (X, or readers of Y) are complete
   // the leader's barriers as seen from either CTA of the pair
   const uint32_t full_l = mapa_shared(smem_addr(full), 0);
-  const uint32_t meta_full_l = mapa_shared(smem_addr(meta_full), 0);
   const uint32_t acc_empty_l = mapa_shared(smem_addr(acc_empty), 0);
 
   if (warp == 0) {
@@ -388,7 +399,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           permute_meta_f16(smem + C::OFF_MSTG + s * C::MSTG_BYTES, smem + C::OFF_MCP + s * C::MCP_BYTES, lane);
           fence_proxy_async_smem();
           __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(meta_full_l + 8u * s);
+          if (lane == 0) mbar_arrive_cluster(full_l + 8u * s);
         }
       }
     }
@@ -420,37 +431,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         if (i >= 2 && !mbar_wait(&acc_empty[b], ((i >> 1) - 1) & 1, abort_flag, err, ERR_WAIT_ACC_FREE)) break;
         tc_fence_after();
         const uint32_t acc = tmem + uint32_t(b * BN);
-        for (int kb = 0; kb < KB; ++kb, ++g) {
-          if (!mbar_wait(&full[s], ph, abort_flag, err, ERR_WAIT_FULL)) {
-            ok = false;
-            break;
-          }
-          if constexpr (!kInt8) {
-            if (!mbar_wait(&meta_full[s], ph, abort_flag, err, ERR_WAIT_META)) {
+        // Stages are issued in groups of kIssueGroup: every barrier of the
+        // group is waited first, then the group's MMAs follow back to back.
+        for (int kb = 0; kb < KB; kb += kIssueGroup) {
+          const int nr = KB - kb < kIssueGroup ? KB - kb : kIssueGroup;
+          int s2 = s;
+          uint32_t ph2 = ph;
+          for (int r = 0; r < nr; ++r) {
+            if (!mbar_wait(&full[s2], ph2, abort_flag, err, ERR_WAIT_FULL)) {
               ok = false;
               break;
             }
+            if (++s2 == STAGES) {
+              s2 = 0;
+              ph2 ^= 1u;
+            }
           }
+          if (!ok) break;
           tc_fence_after();
-          const uint64_t ad = a_desc0 + uint64_t(s) * kAStep;
-          const uint64_t bd = b_desc0 + uint64_t(s) * kBStep;
-          const uint64_t ed = e_desc0 + uint64_t(s) * kEStep;
-          const uint32_t ecol = tmem + C::META_COL + (g & 1) * C::MCOLS;
-          tc_cp_128x128b_pair(ecol, ed);
-          if constexpr (kInt8) tc_cp_128x128b_pair(ecol + 4, ed + (2048 >> 4));
+          for (int r = 0; r < nr; ++r, ++g) {
+            const uint64_t ad = a_desc0 + uint64_t(s) * kAStep;
+            const uint64_t bd = b_desc0 + uint64_t(s) * kBStep;
+            const uint64_t ed = e_desc0 + uint64_t(s) * kEStep;
+            const uint32_t ecol = tmem + C::META_COL + (g & 1) * C::MCOLS;
+            tc_cp_128x128b_pair(ecol, ed);
+            if constexpr (kInt8) tc_cp_128x128b_pair(ecol + 4, ed + (2048 >> 4));
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint64_t adesc = ad + uint64_t((32 * j) >> 4);
-            const uint64_t bdesc = bd + uint64_t(((j >> 1) * (BNH * 128) + (j & 1) * 64) >> 4);
-            const uint32_t e = kInt8 ? ecol + 2 * j : ecol + (j & ~1);
-            const uint32_t sel = kInt8 ? 0u : uint32_t(j & 1);
-            tc_mma_sp_pair<kInt8>(acc, adesc, bdesc, e, instr_desc(kFmt, kCFmt, 256, BN, true, sel),
-                                  (kb | j) != 0 ? 1u : 0u);
-          }
-          tc_commit_pair(&empty[s], 0x3);
-          if (++s == STAGES) {
-            s = 0;
-            ph ^= 1u;
+            for (int j = 0; j < 4; ++j) {
+              const uint64_t adesc = ad + uint64_t((32 * j) >> 4);
+              const uint64_t bdesc = bd + uint64_t(((j >> 1) * (BNH * 128) + (j & 1) * 64) >> 4);
+              const uint32_t e = kInt8 ? ecol + 2 * j : ecol + (j & ~1);
+              const uint32_t sel = kInt8 ? 0u : uint32_t(j & 1);
+              tc_mma_sp_pair<kInt8>(acc, adesc, bdesc, e, instr_desc(kFmt, kCFmt, 256, BN, true, sel),
+                                    ((kb + r) | j) != 0 ? 1u : 0u);
+            }
+            tc_commit_pair(&empty[s], 0x3);
+            if (++s == STAGES) {
+              s = 0;
+              ph ^= 1u;
+            }
           }
         }
         if (!ok) break;
