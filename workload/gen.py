@@ -183,12 +183,15 @@ def tw_tile_counts(N: int, G: int, frac: float):
     return P, Nk, T
 
 
-def _layer_inputs(cfg: Config, seed: int, lname: str, M: int, N: int, K: int, bias: bool) -> dict:
+def _layer_inputs(cfg: Config, seed: int, lname: str, M: int, N: int, K: int, bias: bool, batch: int = 0) -> dict:
     stem = f"{cfg.name}.{lname}"
     wstem = f"{cfg.shared_w}.{lname}" if cfg.shared_w else stem
+    # activations of batch b (b > 0: another data-parallel rank's batch) come from
+    # their own stream; weights, bias and pattern are the model's, the same for all
+    xstem = stem + ".X" if batch == 0 else f"{stem}.X.batch{batch}"
     d: dict = {"M": M, "N": N, "K": K}
     if cfg.kind == "24_s8":
-        d["X"] = uniform_int127(seed, stem + ".X", M * K).reshape(M, K)
+        d["X"] = uniform_int127(seed, xstem, M * K).reshape(M, K)
         w = normal(seed, wstem + ".W", N * K, cfg.w_std).reshape(N, K)
         s = (np.abs(w).max(axis=1) / np.float32(127.0)).astype(np.float32)
         s = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
@@ -212,7 +215,7 @@ def _layer_inputs(cfg: Config, seed: int, lname: str, M: int, N: int, K: int, bi
     to = f32_to_bf16_bits if cfg.kind == "24_bf16" else f32_to_f16
     if cfg.kind == "tw_f32":   # fp32 data; the pattern is selected on the fp16 copy W16
         to = lambda a: np.asarray(a, dtype=np.float32)
-    d["X"] = to(normal(seed, stem + ".X", M * K, cfg.x_std)).reshape(M, K)
+    d["X"] = to(normal(seed, xstem, M * K, cfg.x_std)).reshape(M, K)
     d["W"] = to(normal(seed, wstem + ".W", N * K, cfg.w_std)).reshape(N, K)
     if cfg.kind == "tw_f32":
         d["W16"] = f32_to_f16(d["W"])
@@ -228,21 +231,23 @@ def _layer_inputs(cfg: Config, seed: int, lname: str, M: int, N: int, K: int, bi
     return d
 
 
-def make_inputs(name: str, seed: int = 0, layers=None) -> list:
+def make_inputs(name: str, seed: int = 0, layers=None, batch: int = 0) -> list:
     """Inputs of every layer of configuration ``name`` (list of dicts, one per layer).
 
     Arrays: X [M,K], W [N,K] (dense, before pruning), bias [N] or None, and for
     int8 the per-row weight scale; fp16 arrays are float16, bf16 arrays are
     uint16 bit patterns, int8 arrays are int8.  For tile-wise layers also
     ``G``, ``n_pruned`` and ``k_per_tile`` (workload data: the per-tile kept-row
-    counts drawn from the configured density range).
+    counts drawn from the configured density range).  ``batch`` selects the
+    activation batch (a data-parallel rank's own batch); everything else is
+    the same for every batch.
     """
     cfg = CONFIGS[name]
     out = []
     for (lname, M, N, K, bias) in cfg.layers:
         if layers is not None and lname not in layers:
             continue
-        d = _layer_inputs(cfg, seed, lname, M, N, K, bias)
+        d = _layer_inputs(cfg, seed, lname, M, N, K, bias, batch)
         d["layer"] = lname
         d["kind"] = cfg.kind
         out.append(d)
