@@ -77,3 +77,33 @@ def test_validation_rejects_before_touching_the_device():
     assert L.spgemm_tw_f16_yt(16, 64, 1, ctypes.byref(desc), 16, 32, 64, None, 0, None) == 1  # ldyt < M
     assert L.spgemm_tw_f16_yt(16, 64, 1, ctypes.byref(desc), 18, 64, 64, None, 0, None) == 3  # Yt not 16-B aligned
     assert L.spgemm_tw_f16_yt(16, 64, 1, ctypes.byref(desc), 16, 68, 64, None, 0, None) == 3  # ldyt % 8
+
+
+def test_tw_f32_validation_and_workspace_sizes():
+    """The CUDA-core fp32 tile-wise entry points reject bad arguments on the host."""
+    import structured_sparse_gemm_02_b200 as spg
+    L = spg.lib()
+    # [M, K] inputs are transposed at a pitch rounded up to 4 floats, in 256-byte units
+    assert L.tw_workspace_size_f32(4095, 768, spg.SPG_X_MK) == (4096 * 768 * 4 + 255) // 256 * 256
+    assert L.tw_workspace_size_f32(4096, 768, spg.SPG_X_KM) == 0
+    assert L.tw_workspace_size_f32(0, 768, spg.SPG_X_MK) == 0
+    desc = spg.SpgTwDesc()
+    desc.N, desc.K, desc.Nk, desc.G, desc.T, desc.offsetk_len = 768, 768, 691, 128, 6, 1536
+    for f in ("offsetn", "tile_n0", "tile_kofs", "k_per_tile", "offsetk", "Wc"):
+        setattr(desc, f, 256)
+    d = ctypes.byref(desc)
+    X, W, Y, ws = 4096, 8192, 16384, 32768          # stand-in addresses, 16-byte aligned
+    assert L.spgemm_tw_f32(None, 768, 0, d, W, Y, 768, 64, ws, 1 << 20, None) == 1        # no X
+    assert L.spgemm_tw_f32(X, 768, 5, d, W, Y, 768, 64, ws, 1 << 20, None) == 1           # layout
+    assert L.spgemm_tw_f32(X, 768, 0, d, W, Y, 700, 64, ws, 1 << 20, None) == 1           # ldy < N
+    assert L.spgemm_tw_f32(X, 700, 0, d, W, Y, 768, 64, ws, 1 << 20, None) == 1           # ldx < K
+    assert L.spgemm_tw_f32(X, 768, 0, d, W, Y, 768, 64, None, 0, None) == 1               # no workspace
+    assert L.spgemm_tw_f32(X, 768, 0, d, W, Y, 768, 64, ws, 100, None) == 1               # workspace short
+    assert L.spgemm_tw_f32(X + 4, 64, 1, d, W, Y, 768, 64, None, 0, None) == 3            # Xt rows not 16-B
+    assert L.spgemm_tw_f32(X, 66, 1, d, W, Y, 768, 64, None, 0, None) == 3                # ldx % 4
+    assert L.spgemm_tw_f32(X, 768, 0, d, W + 4, Y, 768, 64, ws, 1 << 20, None) == 3       # Wc32 alignment
+    assert L.spgemm_tw_f32(X, 768, 0, d, W, Y + 2, 768, 64, ws, 1 << 20, None) == 3       # Y alignment
+    assert L.tw_condense_f32(W, 700, d, W, None) == 1                                     # ldw < K
+    assert L.tw_condense_f32(W, 768, d, W + 4, None) == 3                                 # Wc32 alignment
+    desc.G = 64
+    assert L.spgemm_tw_f32(X, 768, 0, d, W, Y, 768, 64, ws, 1 << 20, None) == 1           # G must be 128
