@@ -749,14 +749,31 @@ spg_status launch(const void* X, int64_t ldx, const void* Wv, const uint8_t* met
   return launch_status();
 }
 
-// X rows per pair tile: small batches take narrow tiles, large ones the widest
-// tile whose two accumulators and metadata ring fit in tensor memory.
+// Estimated cost of a launch with X-tile width bn: the rounds of pair tiles the
+// busiest pair runs, each costing its width plus a fixed per-tile share (the
+// epilogue's latency and the pipeline's fill), in units of X rows.  The share
+// of 160 matches the ViT-Base MLP measurements: 224 is faster for
+// 12608 x 3072 x 768 (39.8 against 41.5 us with 192), 192 for
+// 12608 x 768 x 3072 (38.2 against 38.9 us), where 224 leaves the last round
+// a third full.
+int64_t tile_cost(int64_t M, int64_t N, int bn) {
+  const int64_t tiles = ((N + 255) / 256) * ((M + bn - 1) / bn);
+  const int64_t pairs = sm_count() / 2;
+  const int64_t rounds = (tiles + pairs - 1) / pairs;
+  return rounds * (bn + 160);
+}
+
+// X rows per pair tile: small batches take narrow tiles, large ones the wider
+// of 224 (the widest whose two accumulators and metadata ring fit in tensor
+// memory) and 192 by the estimated cost.
 template <bool kInt8, bool kBF16, int OUT>
 spg_status dispatch(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,
                     const float* scale, void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t s,
                     float qscale = 0.f) {
   if (M <= 32) return launch<kInt8, kBF16, 32, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s, qscale);
   if (M <= 128) return launch<kInt8, kBF16, 128, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s, qscale);
+  if (tile_cost(M, N, 192) < tile_cost(M, N, 224))
+    return launch<kInt8, kBF16, 192, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s, qscale);
   return launch<kInt8, kBF16, 224, OUT>(X, ldx, Wv, meta, bias, scale, Y, ldy, M, N, K, s, qscale);
 }
 
