@@ -273,9 +273,23 @@ __device__ __forceinline__ void stage_pair_box16(uint32_t box_saddr, const uint3
   }
 }
 
+// Tile order: the ceil(N/256) x ceil(M/BN) tile grid is walked in bands of
+// `band` consecutive weight-row tiles; inside a band the weight tile varies
+// fastest, so the pairs in flight share X tiles through L2, and a band's
+// compressed weights stay in L2 while every X tile passes by once.  HBM then
+// reads W once and X once per band (the host sizes a band's weights to a
+// fraction of L2; shapes with one band keep the plain n-fastest order).
+__device__ __forceinline__ void tile_coords(int t, int NT, int MT, int band, int& nt, int& mt) {
+  const int per_band = band * MT;
+  const int b = t / per_band;
+  const int r = t - b * per_band;
+  const int w = min(band, NT - b * band);
+  mt = r / w;
+  nt = b * band + (r - mt * w);
+}
+
 // Cluster pairs: pair p = blockIdx.x / 2 computes tiles p, p + gridDim.x/2, ...
-// of the ceil(N/256) x ceil(M/BN) tile grid (n fastest, so the pairs in
-// flight share X tiles through L2).  CTA rank r of the pair loads weight rows
+// in the order of tile_coords.  CTA rank r of the pair loads weight rows
 // [n0 + 128r, +128) and X rows [m0 + r*BN/2, +BN/2); the leader (rank 0)
 // issues the 256 x BN MMAs, which read both CTAs' shared memory and write
 // each CTA's own tensor memory (its 128 weight rows x BN).
@@ -284,7 +298,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     spgemm24_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
                     void* __restrict__ Yp, int64_t ldy, const void* __restrict__ bias,
-                    const float* __restrict__ scale, float qscale, int M, int N, int K, uint32_t* err) {
+                    const float* __restrict__ scale, float qscale, int M, int N, int K, int band,
+                    uint32_t* err) {
   using C = Cfg<kInt8, BN, OUT>;
   constexpr int STAGES = C::STAGES;
   constexpr int BNH = C::BNH;
@@ -305,7 +320,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int KB = K / C::KSTEP;
   const int NT = (N + 255) / 256;
-  const int total = NT * ((M + BN - 1) / BN);
+  const int MT = (M + BN - 1) / BN;
+  const int total = NT * MT;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -350,8 +366,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       uint32_t g = 0;
       bool ok = true;
       for (int t = pair; ok && t < total; t += npairs) {
-        const int n0 = (t % NT) * 256 + 128 * int(rank);
-        const int m0 = (t / NT) * BN + BNH * int(rank);
+        int nt, mt;
+        tile_coords(t, NT, MT, band, nt, mt);
+        const int n0 = nt * 256 + 128 * int(rank);
+        const int m0 = mt * BN + BNH * int(rank);
         for (int kb = 0; kb < KB; ++kb, ++g) {
           const int s = g % STAGES;
           const uint32_t use = g / STAGES;
@@ -500,7 +518,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     uint32_t nyt = 0;     // Y^T: boxes this warp stored so far
     int i = 0;
     for (int t = pair; t < total; t += npairs, ++i) {
-      const int n0 = (t % NT) * 256 + 128 * int(rank), m0 = (t / NT) * BN;
+      int nt, mt;
+      tile_coords(t, NT, MT, band, nt, mt);
+      const int n0 = nt * 256 + 128 * int(rank), m0 = mt * BN;
       const int b = i & 1;
       // the two warps of a pair take the same branch: they meet at the pair barrier below
       const bool got = mbar_wait_warp(&acc_full[b], (i >> 1) & 1, abort_flag, err, ERR_WAIT_ACC);
@@ -743,8 +763,19 @@ spg_status launch(const void* X, int64_t ldx, const void* Wv, const uint8_t* met
   const int64_t pairs_max = resident_pairs(reinterpret_cast<const void*>(kern), C::SMEM, C::THREADS);
   if (pairs_max <= 0) return SPG_ERR_CUDA;
   const int pairs = static_cast<int>(tiles < pairs_max ? tiles : pairs_max);
+  // weight-row tiles per band: their compressed values and metadata take at
+  // most kBandBytes, a fifth of the 126 MB L2 (prefill-sized weights split into
+  // bands; the ViT-sized layers fit in one)
+  constexpr int64_t kBandBytes = int64_t(24) << 20;
+  const int64_t tile_w_bytes = 256 * (K / 2 * es + K / 8);
+  const int64_t nt_all = (N + 255) / 256;
+  int64_t band = kBandBytes / tile_w_bytes;
+  band = band < 1 ? 1 : band > nt_all ? nt_all : band;
+  const int64_t nbands = (nt_all + band - 1) / band;
+  band = (nt_all + nbands - 1) / nbands;  // equal bands (64 tiles: 4 x 16, not 3 x 21 + 1)
   if (launch_pdl(kern, dim3(2 * pairs), dim3(C::THREADS), C::SMEM, stream, tmA, tmB, tmE, tmY, Y, ldy, bias, scale,
-                 qscale, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), err) != cudaSuccess)
+                 qscale, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(band),
+                 err) != cudaSuccess)
     return SPG_ERR_CUDA;
   return launch_status();
 }

@@ -132,6 +132,24 @@ def test_ragged_shapes(spg, kind, M, N, K):
     assert rep["ok"], rep
 
 
+@pytest.mark.parametrize("kind", ["f16", "bf16"])
+def test_banded_tile_order(spg, kind):
+    """Long K puts the weight-row tiles in more than one band of the tile order
+    (K = 4096: 17 + 16 tiles of 256 rows for N = 8292); every output tile,
+    the ragged last row and column tiles included, must still be computed once."""
+    M, N, K = 300, 8292, 4096
+    rng = np.random.default_rng(4096)
+    X = rng.standard_normal((M, K)).astype(np.float32)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    cv = (lambda a: a.astype(np.float16)) if kind == "f16" else gen.f32_to_bf16_bits
+    X, W = cv(X), cv(W)
+    Y = _gemm_case(spg, kind, X, W, None)
+    Wv, meta = s24.compress_24(W, kind)
+    ref = s24.gemm_24_ref(X, Wv, meta, None, kind)
+    rep = compare.check_close(s24.to_f64(Y, kind), ref, K)
+    assert rep["ok"], rep
+
+
 @pytest.mark.parametrize("layer", ["fc1", "fc2"])
 def test_vitb_full_size_sampled(spg, layer):
     d = gen.make_inputs("vitb_mlp_f16", layers=[layer])[0]
