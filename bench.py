@@ -49,6 +49,9 @@ def load_peaks():
 
 PROFILED = {  # workload -> (profile summary, kernel sources whose hash it records)
     "vitb_mlp_f16": ("spgemm24_kernel.vitb_mlp_f16.md", ["spgemm24.cu", "sm100.cuh"]),
+    "vitl_mlp_s8": ("spgemm24_kernel.vitl_mlp_s8.md", ["spgemm24.cu", "sm100.cuh"]),
+    "bf16_prefill": ("spgemm24_kernel.bf16_prefill.md", ["spgemm24.cu", "sm100.cuh"]),
+    "bf16_decode": ("spgemm24_kernel.bf16_decode.md", ["spgemm24.cu", "sm100.cuh"]),
     "tw_bert_f16": ("tw_gemm_kernel.tw_bert_f16.md", ["tw.cu", "sm100.cuh"]),
     "tw_bert_f32": ("tw_gemm_f32_kernel.tw_bert_f32.md", ["tw32.cu", "host.cuh"]),
 }
