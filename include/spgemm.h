@@ -27,6 +27,10 @@
  *    that word.
  *  - Device requirement: compute capability 10.0 (B200, sm_100a); other
  *    devices get SPG_ERR_UNSUPPORTED_DEVICE.
+ *  - An empty batch (M == 0) is valid for every GEMM entry point except
+ *    spgemm_tw_f16_noalloc: the other arguments are validated as usual,
+ *    nothing is launched, SPG_OK is returned, and X, Y (and the workspace)
+ *    may be NULL.
  */
 #ifndef SPGEMM_H_
 #define SPGEMM_H_
@@ -123,7 +127,7 @@ spg_status sparse_compress_24(const void* W, int64_t ldw, void* Wv, uint8_t* met
  *   Wv, meta: as written by sparse_compress_24 for [N, K]
  *   bias [N] or NULL
  *   Y    [M, N], pitch ldy >= N
- * Limits: K % 128 == 0, K >= 128; M, N >= 1 (any value, ragged tiles are
+ * Limits: K % 128 == 0, K >= 128; M >= 0, N >= 1 (any value, ragged tiles are
  * handled); M, N, K < 2^31.  X, Wv, Y 16-byte aligned; ldx and ldy in bytes
  * multiples of 16; meta 16-byte aligned; bias 2-byte aligned.
  * ------------------------------------------------------------------------- */
@@ -283,7 +287,7 @@ size_t tw_workspace_size(int64_t M, int64_t K, int x_layout);
  * [K, M] pitch ldx (SPG_X_KM: the transpose is assumed fused upstream).  Y
  * fp16 [M, N] pitch ldy; every element of Y is written (pruned columns +0).
  * fp32 accumulation, one round-to-nearest-even.
- * Limits: M % 8 == 0 (the [K, M] rows are TMA rows), M >= 8; X and
+ * Limits: M % 8 == 0 (the [K, M] rows are TMA rows), M >= 0; X and
  * workspace 16-byte aligned, ldx a multiple of 8; Y 2-byte aligned, any
  * ldy >= N; ws_bytes >= tw_workspace_size(M, K, x_layout). */
 spg_status spgemm_tw_f16(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Y,

@@ -810,8 +810,9 @@ spg_status dispatch(const void* X, int64_t ldx, const void* Wv, const uint8_t* m
 
 spg_status validate_common(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, void* Y, int64_t ldy,
                            int64_t M, int64_t N, int64_t K, int es, int out_es, int kstep, bool y_transposed = false) {
-  if (!X || !Wv || !meta || !Y) return SPG_ERR_INVALID_ARG;
-  if (M <= 0 || N <= 0 || K <= 0 || ldx < K || ldy < (y_transposed ? M : N)) return SPG_ERR_INVALID_ARG;
+  // M == 0 (an empty batch) is valid: the caller returns SPG_OK without a launch, and X / Y may be NULL
+  if (!Wv || !meta || (M != 0 && (!X || !Y))) return SPG_ERR_INVALID_ARG;
+  if (M < 0 || N <= 0 || K <= 0 || ldx < K || ldy < (y_transposed ? M : N)) return SPG_ERR_INVALID_ARG;
   if (K % kstep || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
     return SPG_ERR_UNSUPPORTED_SHAPE;
   if ((N + 127) / 128 * ((M + 31) / 32) >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
@@ -834,6 +835,7 @@ spg_status spgemm_24_f16(const void* X, int64_t ldx, const void* Wv, const uint8
   spg_status st = validate_common(X, ldx, Wv, meta, Y, ldy, M, N, K, 2, 2, 128);
   if (st != SPG_OK) return st;
   if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;
+  if (M == 0) return SPG_OK;  // empty batch: nothing to compute
   st = check_device();
   if (st != SPG_OK) return st;
   auto s = reinterpret_cast<cudaStream_t>(stream);
@@ -850,6 +852,7 @@ spg_status spgemm_24_f16_gelu(const void* X, int64_t ldx, const void* Wv, const 
   spg_status st = validate_common(X, ldx, Wv, meta, Y, ldy, M, N, K, 2, 2, 128);
   if (st != SPG_OK) return st;
   if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;
+  if (M == 0) return SPG_OK;  // empty batch: nothing to compute
   st = check_device();
   if (st != SPG_OK) return st;
   auto s = reinterpret_cast<cudaStream_t>(stream);
@@ -867,6 +870,7 @@ spg_status spgemm_24_f16_yt(const void* X, int64_t ldx, const void* Wv, const ui
   spg_status st = validate_common(X, ldx, Wv, meta, Yt, ldyt, M, N, K, 2, 2, 128, true);
   if (st != SPG_OK) return st;
   if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;
+  if (M == 0) return SPG_OK;  // empty batch: nothing to compute
   st = check_device();
   if (st != SPG_OK) return st;
   auto s = reinterpret_cast<cudaStream_t>(stream);
@@ -887,6 +891,7 @@ spg_status spgemm_24_s8(const int8_t* X, int64_t ldx, const int8_t* Wv, const ui
   if (out_mode == SPG_OUT_F16 && !scale) return SPG_ERR_INVALID_ARG;
   if (scale && !aligned(scale, 4)) return SPG_ERR_MISALIGNED;
   if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;
+  if (M == 0) return SPG_OK;  // empty batch: nothing to compute
   st = check_device();
   if (st != SPG_OK) return st;
   auto s = reinterpret_cast<cudaStream_t>(stream);
@@ -908,6 +913,7 @@ spg_status spgemm_24_s8_q(const int8_t* X, int64_t ldx, const int8_t* Wv, const 
   if (st != SPG_OK) return st;
   if (!aligned(scale, 4)) return SPG_ERR_MISALIGNED;
   if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;
+  if (M == 0) return SPG_OK;  // empty batch: nothing to compute
   st = check_device();
   if (st != SPG_OK) return st;
   auto s = reinterpret_cast<cudaStream_t>(stream);

@@ -705,16 +705,18 @@ spg_status launch_gemm(const uint16_t* xt, int64_t ldt, const spg_tw_desc* desc,
 // spgemm_tw_f16 (Y [M][N], y_nm false) and spgemm_tw_f16_yt (Y^T [N][M]).
 spg_status run(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Y, int64_t ldy, int64_t M,
                void* workspace, size_t ws_bytes, spg_stream_t stream, bool y_nm) {
-  if (!X || !desc || !Y) return SPG_ERR_INVALID_ARG;
+  // M == 0 (an empty batch) is valid: SPG_OK without a launch, and X / Y / workspace may be NULL
+  if (!desc || (M != 0 && (!X || !Y))) return SPG_ERR_INVALID_ARG;
   if (x_layout != SPG_X_MK && x_layout != SPG_X_KM) return SPG_ERR_INVALID_ARG;
   const int64_t N = desc->N, K = desc->K;
-  if (M <= 0 || N <= 0 || K <= 0 || ldy < (y_nm ? M : N)) return SPG_ERR_INVALID_ARG;
+  if (M < 0 || N <= 0 || K <= 0 || ldy < (y_nm ? M : N)) return SPG_ERR_INVALID_ARG;
   if (desc->G != kG || desc->T <= 0 || desc->offsetk_len <= 0 || desc->offsetk_len % kKBlock) return SPG_ERR_INVALID_ARG;
   if (!desc->offsetn || !desc->tile_n0 || !desc->tile_kofs || !desc->offsetk || !desc->Wc) return SPG_ERR_INVALID_ARG;
   if (x_layout == SPG_X_MK ? ldx < K : ldx < M) return SPG_ERR_INVALID_ARG;
   if (M % 8 || M >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(X, 16) || !aligned(Y, 2) || ldx % 8) return SPG_ERR_MISALIGNED;
   if (y_nm && (!aligned(Y, 16) || ldy % 8)) return SPG_ERR_MISALIGNED;
+  if (M == 0) return SPG_OK;  // empty batch: nothing to compute
   if (x_layout == SPG_X_MK) {
     if (!workspace || ws_bytes < tw_workspace_size(M, K, x_layout)) return SPG_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return SPG_ERR_MISALIGNED;

@@ -324,13 +324,15 @@ spg_status spgemm_tw_f32(const float* X, int64_t ldx, int x_layout, const spg_tw
   using namespace spg::tw32;
   spg_status st = check_desc(desc);
   if (st != SPG_OK) return st;
-  if (!X || !Wc32 || !Y) return SPG_ERR_INVALID_ARG;
+  // M == 0 (an empty batch) is valid: SPG_OK without a launch, and X / Y / workspace may be NULL
+  if (!Wc32 || (M != 0 && (!X || !Y))) return SPG_ERR_INVALID_ARG;
   if (x_layout != SPG_X_MK && x_layout != SPG_X_KM) return SPG_ERR_INVALID_ARG;
   const int64_t N = desc->N, K = desc->K;
-  if (M <= 0 || ldy < N || (x_layout == SPG_X_MK ? ldx < K : ldx < M)) return SPG_ERR_INVALID_ARG;
+  if (M < 0 || ldy < N || (x_layout == SPG_X_MK ? ldx < K : ldx < M)) return SPG_ERR_INVALID_ARG;
   if (M >= (int64_t(1) << 31) || int64_t(desc->T) * ((M + 63) / 64) >= (int64_t(1) << 31))
     return SPG_ERR_UNSUPPORTED_SHAPE;  // one block per (tile, row block)
   if (!aligned(X, 4) || !aligned(Wc32, 16) || !aligned(Y, 4)) return SPG_ERR_MISALIGNED;
+  if (M == 0) return SPG_OK;  // empty batch: nothing to compute
   if (x_layout == SPG_X_KM) {
     if (!aligned(X, 16) || ldx % 4) return SPG_ERR_MISALIGNED;  // 16-byte copies of Xt rows
   } else {

@@ -107,3 +107,33 @@ def test_tw_f32_validation_and_workspace_sizes():
     assert L.tw_condense_f32(W, 768, d, W + 4, None) == 3                                 # Wc32 alignment
     desc.G = 64
     assert L.spgemm_tw_f32(X, 768, 0, d, W, Y, 768, 64, ws, 1 << 20, None) == 1           # G must be 128
+
+
+def test_empty_batch_is_a_no_op():
+    """M == 0 returns SPG_OK before anything touches the device (X, Y and the
+    workspace may be NULL); the other arguments are still validated."""
+    import structured_sparse_gemm_02_b200 as spg
+    L = spg.lib()
+    Wv, meta, sc = 4096, 8192, 12288                   # stand-in addresses, 16-byte aligned
+    assert L.spgemm_24_f16(None, 256, Wv, meta, None, None, 256, 0, 256, 256, 0, None) == 0
+    assert L.spgemm_24_f16_gelu(None, 256, Wv, meta, None, None, 256, 0, 256, 256, 1, None) == 0
+    assert L.spgemm_24_f16_yt(None, 256, Wv, meta, None, None, 0, 0, 256, 256, 0, None) == 0
+    assert L.spgemm_24_s8(None, 256, Wv, meta, sc, None, None, 256, 0, 0, 256, 256, None) == 0
+    assert L.spgemm_24_s8_q(None, 256, Wv, meta, sc, None, ctypes.c_float(1.0), 0, None, 256, 0, 256, 256,
+                            None) == 0
+    assert L.spgemm_24_f16(None, 256, Wv, meta, None, None, 256, 0, 256, 192, 0, None) == 2   # K % 128
+    assert L.spgemm_24_f16(None, 256, None, meta, None, None, 256, 0, 256, 256, 0, None) == 1  # no Wv
+    assert L.spgemm_24_f16(None, 256, Wv, meta, None, None, 256, -1, 256, 256, 0, None) == 1  # M < 0
+    assert L.spgemm_24_s8(None, 256, Wv, meta, None, None, None, 256, 0, 0, 256, 256, None) == 1  # scale
+    desc = spg.SpgTwDesc()
+    desc.N, desc.K, desc.Nk, desc.G, desc.T, desc.offsetk_len = 768, 768, 691, 128, 6, 1536
+    for f in ("offsetn", "tile_n0", "tile_kofs", "k_per_tile", "offsetk", "Wc"):
+        setattr(desc, f, 256)
+    d = ctypes.byref(desc)
+    assert L.tw_workspace_size(0, 768, spg.SPG_X_MK) == 0
+    assert L.spgemm_tw_f16(None, 768, spg.SPG_X_MK, d, None, 768, 0, None, 0, None) == 0
+    assert L.spgemm_tw_f16_yt(None, 0, spg.SPG_X_KM, d, None, 0, 0, None, 0, None) == 0
+    assert L.spgemm_tw_f32(None, 768, spg.SPG_X_MK, d, Wv, None, 768, 0, None, 0, None) == 0
+    assert L.spgemm_tw_f16(None, 768, spg.SPG_X_MK, d, None, 700, 0, None, 0, None) == 1      # ldy < N
+    # the entry point without allocation keeps M >= 8 (its limits are its own)
+    assert L.spgemm_tw_f16_noalloc(None, 768, d, None, 768, 0, None) == 1

@@ -132,6 +132,18 @@ def test_ragged_shapes(spg, kind, M, N, K):
     assert rep["ok"], rep
 
 
+def test_empty_batch_through_the_binding(spg):
+    """An empty batch (M = 0, a zero-size torch tensor) is a no-op with a [0, N] result."""
+    import torch
+    W = (torch.randn(256, 512, device="cuda") * 0.02).half()
+    Wv, meta = spg.sparse_compress_24(W)
+    Y = spg.spgemm_24_f16(torch.empty((0, 512), dtype=torch.float16, device="cuda"), Wv, meta)
+    assert tuple(Y.shape) == (0, 256)
+    Yt = spg.spgemm_24_f16_yt(torch.empty((0, 512), dtype=torch.float16, device="cuda"), Wv, meta)
+    assert tuple(Yt.shape) == (256, 0)
+    assert spg.check_device_error() == 0
+
+
 @pytest.mark.parametrize("kind", ["f16", "bf16"])
 def test_banded_tile_order(spg, kind):
     """Long K puts the weight-row tiles in more than one band of the tile order
