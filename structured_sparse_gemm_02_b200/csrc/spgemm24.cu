@@ -816,6 +816,7 @@ spg_status validate_common(const void* X, int64_t ldx, const void* Wv, const uin
   if (K % kstep || M >= (int64_t(1) << 31) || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31))
     return SPG_ERR_UNSUPPORTED_SHAPE;
   if ((N + 127) / 128 * ((M + 31) / 32) >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return SPG_OK;  // nothing is read or written: pointers and pitches need no alignment
   if (!aligned(X, 16) || !aligned(Wv, 16) || !aligned(meta, 16) || !aligned(Y, 16)) return SPG_ERR_MISALIGNED;
   if ((ldx * es) % 16 || (ldy * out_es) % 16) return SPG_ERR_MISALIGNED;
   return SPG_OK;

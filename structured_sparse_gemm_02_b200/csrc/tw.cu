@@ -713,10 +713,10 @@ spg_status run(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc
   if (desc->G != kG || desc->T <= 0 || desc->offsetk_len <= 0 || desc->offsetk_len % kKBlock) return SPG_ERR_INVALID_ARG;
   if (!desc->offsetn || !desc->tile_n0 || !desc->tile_kofs || !desc->offsetk || !desc->Wc) return SPG_ERR_INVALID_ARG;
   if (x_layout == SPG_X_MK ? ldx < K : ldx < M) return SPG_ERR_INVALID_ARG;
+  if (M == 0) return SPG_OK;  // empty batch: nothing is read or written
   if (M % 8 || M >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(X, 16) || !aligned(Y, 2) || ldx % 8) return SPG_ERR_MISALIGNED;
   if (y_nm && (!aligned(Y, 16) || ldy % 8)) return SPG_ERR_MISALIGNED;
-  if (M == 0) return SPG_OK;  // empty batch: nothing to compute
   if (x_layout == SPG_X_MK) {
     if (!workspace || ws_bytes < tw_workspace_size(M, K, x_layout)) return SPG_ERR_INVALID_ARG;
     if (!aligned(workspace, 16)) return SPG_ERR_MISALIGNED;

@@ -331,8 +331,8 @@ spg_status spgemm_tw_f32(const float* X, int64_t ldx, int x_layout, const spg_tw
   if (M < 0 || ldy < N || (x_layout == SPG_X_MK ? ldx < K : ldx < M)) return SPG_ERR_INVALID_ARG;
   if (M >= (int64_t(1) << 31) || int64_t(desc->T) * ((M + 63) / 64) >= (int64_t(1) << 31))
     return SPG_ERR_UNSUPPORTED_SHAPE;  // one block per (tile, row block)
+  if (M == 0) return SPG_OK;  // empty batch: nothing is read or written
   if (!aligned(X, 4) || !aligned(Wc32, 16) || !aligned(Y, 4)) return SPG_ERR_MISALIGNED;
-  if (M == 0) return SPG_OK;  // empty batch: nothing to compute
   if (x_layout == SPG_X_KM) {
     if (!aligned(X, 16) || ldx % 4) return SPG_ERR_MISALIGNED;  // 16-byte copies of Xt rows
   } else {

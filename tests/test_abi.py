@@ -121,6 +121,8 @@ def test_empty_batch_is_a_no_op():
     assert L.spgemm_24_s8(None, 256, Wv, meta, sc, None, None, 256, 0, 0, 256, 256, None) == 0
     assert L.spgemm_24_s8_q(None, 256, Wv, meta, sc, None, ctypes.c_float(1.0), 0, None, 256, 0, 256, 256,
                             None) == 0
+    # zero-size torch tensors report a row stride of 1 ([N, 0] outputs, [K, 0] inputs): not checked
+    assert L.spgemm_24_f16_yt(None, 256, Wv, meta, None, None, 1, 0, 256, 256, 0, None) == 0
     assert L.spgemm_24_f16(None, 256, Wv, meta, None, None, 256, 0, 256, 192, 0, None) == 2   # K % 128
     assert L.spgemm_24_f16(None, 256, None, meta, None, None, 256, 0, 256, 256, 0, None) == 1  # no Wv
     assert L.spgemm_24_f16(None, 256, Wv, meta, None, None, 256, -1, 256, 256, 0, None) == 1  # M < 0
@@ -132,7 +134,8 @@ def test_empty_batch_is_a_no_op():
     d = ctypes.byref(desc)
     assert L.tw_workspace_size(0, 768, spg.SPG_X_MK) == 0
     assert L.spgemm_tw_f16(None, 768, spg.SPG_X_MK, d, None, 768, 0, None, 0, None) == 0
-    assert L.spgemm_tw_f16_yt(None, 0, spg.SPG_X_KM, d, None, 0, 0, None, 0, None) == 0
+    assert L.spgemm_tw_f16_yt(None, 1, spg.SPG_X_KM, d, None, 1, 0, None, 0, None) == 0
+    assert L.spgemm_tw_f32(None, 1, spg.SPG_X_KM, d, Wv, None, 768, 0, None, 0, None) == 0
     assert L.spgemm_tw_f32(None, 768, spg.SPG_X_MK, d, Wv, None, 768, 0, None, 0, None) == 0
     assert L.spgemm_tw_f16(None, 768, spg.SPG_X_MK, d, None, 700, 0, None, 0, None) == 1      # ldy < N
     # the entry point without allocation keeps M >= 8 (its limits are its own)
