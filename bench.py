@@ -564,8 +564,14 @@ def measure_e2e(spg, layers, kind, args, stream):
 # CPU oracle (baseline leg and reference arm)
 
 def oracle_step(inputs, kind, rows_frac=1.0):
-    """Run the oracle over (a row sample of) every layer; returns dense-eq FLOPs computed."""
-    from oracle import sparse24 as s24, tilewise as tw
+    """Run the plain C++ oracle over (a row sample of) every layer; returns dense-eq FLOPs computed.
+
+    2:4 layers: selection and compression, then the fp64 (fp16 / bf16) or exact
+    int64 (int8, with the fp32 dequantisation) product over the masked weight.
+    Tile-wise layers: the numpy oracle's reorganisation (its exact integer
+    norms), then the C++ expansion to a dense weight and its fp64 product.
+    The int8 chain's GELU + quantisation step is the numpy oracle's."""
+    from oracle import native, sparse24 as s24, tilewise as tw
     flops = 0.0
     prev = None
     for d in inputs:
@@ -574,26 +580,29 @@ def oracle_step(inputs, kind, rows_frac=1.0):
         if rows_frac < 1.0:
             rows = np.arange(0, M, max(1, int(round(1.0 / rows_frac))))
             M = len(rows)
-        if kind == "tw_f16":
-            r = tw.tw_reorganize(d["W"], d["G"], d["n_pruned"], d["k_per_tile"])
-            tw.tw_gemm_ref(d["X"], r, rows=rows)
-        elif kind == "tw_f32":
-            r = tw.tw_condense_values(d["W"], tw.tw_reorganize(d["W16"], d["G"], d["n_pruned"], d["k_per_tile"]))
-            tw.tw_gemm_ref(d["X"], r, rows=rows)
+        if kind in ("tw_f16", "tw_f32"):
+            r = tw.tw_reorganize(d["W16"] if kind == "tw_f32" else d["W"], d["G"], d["n_pruned"], d["k_per_tile"])
+            if kind == "tw_f32":
+                r = tw.tw_condense_values(d["W"], r)
+            offsetn, kofs, kk, offsetk, Wc = native.tw_descriptor(r)
+            if kind == "tw_f32":
+                Wc = np.ascontiguousarray(Wc.transpose(0, 2, 1))
+            Wd = native.tw_expand(d["N"], d["K"], offsetn, kofs, kk, offsetk, Wc)
+            native.gemm_f64(d["X"], Wd, rows=rows)
         elif kind == "24_s8":
-            Wv, meta = s24.compress_24(d["W"], "s8")
+            Wv, meta = native.compress_24(d["W"], "s8")
             if d["X"] is None:          # chained: the previous layer's int8 output (same rows)
-                acc = s24.gemm_24_s8_ref(prev, Wv, meta)
+                acc = native.gemm_24_s8_ref(prev, Wv, meta)
             else:
-                acc = s24.gemm_24_s8_ref(d["X"], Wv, meta, rows=rows)
+                acc = native.gemm_24_s8_ref(d["X"], Wv, meta, rows=rows)
             if d.get("qscale") is not None:
                 prev = s24.quantize_s8(acc, d["scale"], d.get("bias"), d["qscale"], True)
             else:
-                s24.dequant_s8(acc, d["scale"], d.get("bias"))
+                native.dequant_s8(acc, d["scale"], d.get("bias"))
         else:
             k = DTYPE_NAME[kind]
-            Wv, meta = s24.compress_24(d["W"], k)
-            s24.gemm_24_ref(d["X"], Wv, meta, d.get("bias"), k, rows=rows)
+            Wv, meta = native.compress_24(d["W"], k)
+            native.gemm_24_ref(d["X"], Wv, meta, d.get("bias"), k, rows=rows)
         flops += 2.0 * M * d["N"] * d["K"]
     return flops
 
@@ -610,8 +619,8 @@ def time_oracle(workload, budget_s):
     inputs = gen.make_inputs(workload)
     frac = 1.0
     total = sum(2.0 * d["M"] * d["N"] * d["K"] for d in inputs)
-    if total > 2e11:
-        frac = 2e11 / total
+    if total > 1.2e11:                 # about 5 s a pass on 16 host cores
+        frac = 1.2e11 / total
     t0 = time.perf_counter()
     flops = oracle_step(inputs, cfg.kind, frac)
     dt = time.perf_counter() - t0
@@ -622,7 +631,8 @@ def time_oracle(workload, budget_s):
     dt = time.perf_counter() - t0
     sample = (f"{reps} pass(es) of the oracle over "
               + ("all rows" if frac >= 1.0 else f"every {int(round(1 / frac))}th row")
-              + f" of every layer of {workload} (fp64 numpy, includes compression)")
+              + f" of every layer of {workload} (plain C++ oracle: fp64 / exact int64 sequential sums,"
+              " OpenMP over rows; includes compression)")
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
             "sample": sample, "seconds": dt}
 
