@@ -113,6 +113,10 @@ def test_tiny_config_parity(spg):
     ref = s24.gemm_24_ref(d["X"], Wv, meta, None, "f16")
     rep = compare.check_close(Y, ref, d["K"])
     assert rep["ok"], rep
+    from oracle import native
+    Wv_c, meta_c = native.compress_24(d["W"], "f16")
+    rep = compare.check_close(Y, native.gemm_24_ref(d["X"], Wv_c, meta_c, None, "f16"), d["K"])
+    assert rep["ok"], rep
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 128, 128), (15, 200, 256), (17, 129, 384), (129, 300, 640),
@@ -215,6 +219,13 @@ def test_vitl_int8_full_bit_exact(spg):
     bias = (rng.standard_normal(d["N"]) * 0.01).astype(np.float16)
     Y16b = _s8_case(spg, d["X"], d["W"], d["scale"], bias, spg.SPG_OUT_F16)
     assert np.array_equal(Y16b.view(np.uint16), s24.dequant_s8(acc, d["scale"], bias).view(np.uint16))
+    # the plain C++ oracle gives the same integers and codes: its own selection,
+    # int64 sums and fp32 dequantisation
+    from oracle import native
+    Wv_c, meta_c = native.compress_24(d["W"], "s8")
+    acc_c = native.gemm_24_s8_ref(d["X"], Wv_c, meta_c)
+    assert np.array_equal(Y32.astype(np.int64), acc_c)
+    assert np.array_equal(Y16b.view(np.uint16), native.dequant_s8(acc_c, d["scale"], bias).view(np.uint16))
 
 
 def test_bf16_decode_and_prefill_sampled(spg):
