@@ -51,6 +51,18 @@ spg_status check_device(int* dev_out) {
   return st == 1 ? SPG_OK : SPG_ERR_UNSUPPORTED_DEVICE;
 }
 
+int sm_count() {
+  static int cached[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int v = __atomic_load_n(&cached[dev], __ATOMIC_ACQUIRE);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+    __atomic_store_n(&cached[dev], v, __ATOMIC_RELEASE);
+  }
+  return v;
+}
+
 uint32_t* device_error_word() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;

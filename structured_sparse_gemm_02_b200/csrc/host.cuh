@@ -18,6 +18,9 @@ spg_status check_device(int* dev_out = nullptr);
 // Device address of the library's error word on the current device.
 uint32_t* device_error_word();
 
+// Number of SMs of the current device (cached per device; 148 if the query fails).
+int sm_count();
+
 // 2-D tiled tensor map over a row-major matrix of `rows` x `cols` elements of
 // `esize` bytes with a row pitch of `pitch_bytes`; the box is box_cols x
 // box_rows.  Returns false if the driver rejects the description.

@@ -34,6 +34,7 @@
 
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "host.cuh"
 #include "sm100.cuh"
@@ -698,25 +699,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   }
 }
 
-int sm_count() {
-  static int cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int v = 148;
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = v;
-  }
-  return cached[dev];
-}
-
-// Cluster pairs of `kern` that fit on the device at once (cached per kernel and device).
+// Cluster pairs of `kern` that fit on the device at once (cached per kernel and
+// device; the cache is shared by every host thread, under a lock).
 int resident_pairs(const void* kern, int smem, int threads) {
   struct Entry { const void* k; int dev; int n; };
+  static std::mutex mu;
   static Entry cache[64];
   static int used = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  std::lock_guard<std::mutex> lk(mu);
   for (int i = 0; i < used; ++i)
     if (cache[i].k == kern && cache[i].dev == dev) return cache[i].n;
   cudaLaunchConfig_t cfg = {};

@@ -626,18 +626,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-int sm_count() {
-  static int cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int v = 148;
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = v;
-  }
-  return cached[dev];
-}
-
 // The GEMM's dynamic shared-memory limit, raised once per device.
 bool smem_attr_set() {
   static int done[64];

@@ -256,18 +256,6 @@ spg_status check_desc(const spg_tw_desc* desc) {
   return SPG_OK;
 }
 
-int sm_count() {
-  static int cached[64];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (!cached[dev]) {
-    int v = 148;
-    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    cached[dev] = v;
-  }
-  return cached[dev];
-}
-
 // Both GEMM variants' dynamic shared-memory limits, raised once per device.
 bool smem_attr_set() {
   static int done[64];
