@@ -20,6 +20,7 @@ import json
 import math
 import os
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -106,7 +107,9 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{os.environ.get('RANK', '0')}.csv")
+        # raw samples (the JSON line carries their summary); SPG_CLOCKS_DIR keeps them elsewhere
+        out = os.environ.get("SPG_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out, f"spg_clocks_rank{os.environ.get('RANK', '0')}.csv")
 
     def start(self):
         try:
