@@ -47,6 +47,8 @@ def lib() -> ctypes.CDLL:
             "orc_gemm24_s8": [p, i64, i64, p, p, i64, p, i64, p],
             "orc_dequant_s8": [p, i64, i64, p, p, p],
             "orc_f32_to_f16": [p, i64, p],
+            "orc_gelu_f64": [p, i64, p],
+            "orc_quantize_s8": [p, i64, i64, p, p, ctypes.c_float, i32, p],
             "orc_tw_expand": [i64, i64, i32, i64, i32, p, p, p, p, p, i32, p],
         }
         for name, args in sig.items():
@@ -143,6 +145,24 @@ def dequant_s8(acc, scale, bias=None):
     Y = np.empty((R, N), dtype=np.float16)
     assert lib().orc_dequant_s8(_ptr(acc), R, N, _ptr(scale), _ptr(b), _ptr(Y)) == 0
     return Y
+
+
+def gelu_f64(v):
+    v = _c(np.asarray(v, dtype=np.float64))
+    y = np.empty_like(v)
+    assert lib().orc_gelu_f64(_ptr(v), v.size, _ptr(y)) == 0
+    return y
+
+
+def quantize_s8(acc, scale, bias, qscale, gelu):
+    """int8 codes of the fixed-point epilogue (see oracle.cpp)."""
+    acc = _c(np.asarray(acc, dtype=np.int64))
+    scale = _c(np.asarray(scale, dtype=np.float32))
+    b = None if bias is None else _c(np.asarray(bias, dtype=np.float16))
+    R, N = acc.shape
+    Yq = np.empty((R, N), dtype=np.int8)
+    assert lib().orc_quantize_s8(_ptr(acc), R, N, _ptr(scale), _ptr(b), float(qscale), int(bool(gelu)), _ptr(Yq)) == 0
+    return Yq
 
 
 def f32_to_f16(x):

@@ -15,6 +15,8 @@
 //  * the dense product over the explicitly masked weight in fp64 (fp16 / bf16
 //    inputs), and in exact integers (int8 inputs) followed by the fp32
 //    dequantisation y = fp16(fp32(acc) * scale[n] [+ fp32(bias[n])]);
+//  * the fixed-point epilogue of the int8 chain (GELU in a fixed fp32
+//    operation order, then the int8 quantiser) and GELU in fp64;
 //  * the tile-wise expansion back to a dense weight ("Accelerating Sparse DNN
 //    Models without Hardware-Support via Tile-Wise Sparsity", slides
 //    "Re-organize" and "Run-time": C[offsetn[n]] += A[offsetk[k]] * B) and
@@ -233,6 +235,62 @@ int orc_dequant_s8(const int64_t* acc, int64_t rows, int64_t N, const float* sca
       float v = float(acc[i * N + n]) * scale[n];
       if (bias) v = v + float(f16_value(bias[n]));
       Y[i * N + n] = f32_to_f16_rne(v);
+    }
+  return 0;
+}
+
+// The activation between the two layers of a ViT MLP block (the models the
+// 2:4 scheme compresses; the pages do not spell it out): GELU(v) = v Phi(v) =
+// 0.5 v (1 + erf(v / sqrt 2)), exact form, in fp64 with the C library's erf.
+int orc_gelu_f64(const double* v, int64_t n, double* y) {
+  for (int64_t i = 0; i < n; ++i) y[i] = 0.5 * v[i] * (1.0 + std::erf(v[i] / std::sqrt(2.0)));
+  return 0;
+}
+
+// The fixed-point epilogue that feeds the next int8 layer, every step one IEEE
+// fp32 operation in this order (built without FMA contraction):
+//   v = fp32(acc) * scale[n]  [ + fp32(bias[n]) ]
+//   [ v = GELU(v) with erf from Abramowitz & Stegun 7.1.28:
+//       u = v * 0.70710677; a = min(|u|, 4);
+//       p = ((((((a6 a + a5) a + a4) a + a3) a + a2) a + a1) a) + 1;
+//       p16 = p^16 by four squarings; r = 1 / p16 by three Newton steps
+//       r = r (2 - p16 r) from the fp32 whose bits are 0x7EF00000 - bits(p16);
+//       erf(u) = sign(u) (1 - r); GELU = (0.5 v) (1 + erf(u)) ]
+//   q = clamp(rne(v * qscale), -127, 127)
+int orc_quantize_s8(const int64_t* acc, int64_t rows, int64_t N, const float* scale, const uint16_t* bias,
+                    float qscale, int gelu, int8_t* Yq) {
+  const float a1 = 0.0705230784f, a2 = 0.0422820123f, a3 = 0.0092705272f, a4 = 0.0001520143f,
+              a5 = 0.0002765672f, a6 = 0.0000430638f;
+  for (int64_t i = 0; i < rows; ++i)
+    for (int64_t n = 0; n < N; ++n) {
+      float v = float(acc[i * N + n]) * scale[n];
+      if (bias) v = v + float(f16_value(bias[n]));
+      if (gelu) {
+        const float u = v * 0.70710677f;
+        const float a = std::fabs(u) < 4.0f ? std::fabs(u) : 4.0f;
+        float h = a6;
+        h = h * a + a5;
+        h = h * a + a4;
+        h = h * a + a3;
+        h = h * a + a2;
+        h = h * a + a1;
+        const float p = h * a + 1.0f;
+        const float p2 = p * p, p4 = p2 * p2, p8 = p4 * p4, p16 = p8 * p8;
+        uint32_t bits;
+        std::memcpy(&bits, &p16, 4);
+        bits = 0x7EF00000u - bits;
+        float r;
+        std::memcpy(&r, &bits, 4);
+        for (int it = 0; it < 3; ++it) r = r * (2.0f - p16 * r);
+        const float e = 1.0f - r;
+        v = (0.5f * v) * (1.0f + (u < 0.0f ? -e : e));
+      }
+      const float t = v * qscale;
+      // round to nearest, ties to even, then clamp
+      float rq = std::floor(t);
+      const float fr = t - rq;
+      if (fr > 0.5f || (fr == 0.5f && std::fmod(rq, 2.0f) != 0.0f)) rq += 1.0f;
+      Yq[i * N + n] = int8_t(rq > 127.0f ? 127 : rq < -127.0f ? -127 : int(rq));
     }
   return 0;
 }

@@ -166,3 +166,32 @@ def test_tw_expand_and_product_match_numpy():
     *_, Wc32 = native.tw_descriptor(r32)
     Wd32 = native.tw_expand(N, K, offsetn, kofs, kk, offsetk, np.ascontiguousarray(Wc32.transpose(0, 2, 1)))
     assert np.array_equal(Wd32, tw.tw_expand(r32).astype(np.float64))
+
+
+def test_fixed_point_epilogue_matches_numpy_bit_for_bit():
+    """The int8 chain's epilogue (fp32 A&S GELU and the int8 quantiser), stated
+    independently in C++ and in numpy, gives the same codes; so does the plain
+    dequantisation path without GELU.  Inputs span the clamp at +-127, the
+    GELU's |u| >= 4 plateau and exact .5 ties of the rounding."""
+    rng = np.random.default_rng(21)
+    R, N = 64, 512
+    acc = rng.integers(-2_000_000, 2_000_000, (R, N)).astype(np.int64)
+    acc[0, :8] = [0, 1, -1, 2 ** 23, -(2 ** 23), 7, -7, 12345]
+    scale = (np.abs(rng.standard_normal(N)) * 2e-6 + 1e-7).astype(np.float32)
+    bias = (rng.standard_normal(N) * 0.01).astype(np.float16)
+    for qscale in (1.0, 31.75, 200.0):
+        for gelu in (False, True):
+            for b in (None, bias):
+                got = native.quantize_s8(acc, scale, b, qscale, gelu)
+                want = s24.quantize_s8(acc, scale, b, qscale, gelu)
+                assert np.array_equal(got, want), (qscale, gelu, b is None)
+    # exact .5 ties: v * qscale lands on k + 0.5 (scale 0.5, qscale 1)
+    ties = np.arange(-20, 21, dtype=np.int64)[None, :]
+    half = np.full(ties.shape[1], 0.5, dtype=np.float32)
+    assert np.array_equal(native.quantize_s8(ties, half, None, 1.0, False),
+                          s24.quantize_s8(ties, half, None, 1.0, False))
+
+
+def test_gelu_f64_matches_numpy():
+    v = np.linspace(-8, 8, 4001)
+    assert np.allclose(native.gelu_f64(v), s24.gelu_ref(v), rtol=1e-15, atol=1e-15)
