@@ -50,6 +50,7 @@ def lib() -> ctypes.CDLL:
             "orc_gelu_f64": [p, i64, p],
             "orc_quantize_s8": [p, i64, i64, p, p, ctypes.c_float, i32, p],
             "orc_tw_expand": [i64, i64, i32, i64, i32, p, p, p, p, p, i32, p],
+            "orc_tw_reorganize": [p, i64, i64, i32, i64, p, p, p, p, p],
         }
         for name, args in sig.items():
             f = getattr(L, name)
@@ -170,6 +171,23 @@ def f32_to_f16(x):
     y = np.empty(x.shape, dtype=np.float16)
     assert lib().orc_f32_to_f16(_ptr(x), x.size, _ptr(y)) == 0
     return y
+
+
+def tw_reorganize(W, n_pruned, k_per_tile, G=128):
+    """Tile-wise descriptor arrays of a dense fp16 W [N, K] (see oracle.cpp):
+    (offsetn, tile_kofs, offsetk, Wc fp16 [blocks, G, 64])."""
+    W = _c(np.asarray(W, dtype=np.float16))
+    N, K = W.shape
+    kpt = _c(np.asarray(k_per_tile, dtype=np.int32))
+    T = len(kpt)
+    kpad = int(sum((int(k) + 63) // 64 * 64 for k in kpt))
+    offsetn = np.empty(N - n_pruned, dtype=np.int32)
+    tile_kofs = np.empty(T + 1, dtype=np.int32)
+    offsetk = np.empty(kpad, dtype=np.int32)
+    Wc = np.empty((kpad // 64, G, 64), dtype=np.float16)
+    assert lib().orc_tw_reorganize(_ptr(W), N, K, G, int(n_pruned), _ptr(kpt), _ptr(offsetn), _ptr(tile_kofs),
+                                   _ptr(offsetk), _ptr(Wc)) == 0
+    return offsetn, tile_kofs, offsetk, Wc
 
 
 def tw_expand(N, K, offsetn, tile_kofs, k_per_tile, offsetk, Wc, G=128):

@@ -17,7 +17,8 @@
 //    dequantisation y = fp16(fp32(acc) * scale[n] [+ fp32(bias[n])]);
 //  * the fixed-point epilogue of the int8 chain (GELU in a fixed fp32
 //    operation order, then the int8 quantiser) and GELU in fp64;
-//  * the tile-wise expansion back to a dense weight ("Accelerating Sparse DNN
+//  * the tile-wise reorganisation with exact integer norms, and the expansion
+//    back to a dense weight ("Accelerating Sparse DNN
 //    Models without Hardware-Support via Tile-Wise Sparsity", slides
 //    "Re-organize" and "Run-time": C[offsetn[n]] += A[offsetk[k]] * B) and
 //    its fp64 product.
@@ -25,6 +26,7 @@
 // Every output element is one sequential sum over k in index order, so the
 // result does not depend on the thread count (OpenMP splits output rows).
 // Build: g++ -O3 -ffp-contract=off -fopenmp -shared -fPIC (oracle/native.py).
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -298,6 +300,78 @@ int orc_quantize_s8(const int64_t* acc, int64_t rows, int64_t N, const float* sc
 // fp32 -> fp16 bits (round to nearest even), exposed for its own test.
 int orc_f32_to_f16(const float* x, int64_t n, uint16_t* y) {
   for (int64_t i = 0; i < n; ++i) y[i] = f32_to_f16_rne(x[i]);
+  return 0;
+}
+
+// Tile-wise reorganisation ("Accelerating Sparse DNN Models without
+// Hardware-Support via Tile-Wise Sparsity", slides "Tile-Wise Sparsity",
+// "Re-organize", "Preprocessed"), with the readings where the slides are
+// silent: columns of B = W^T (rows n of W) are pruned globally by smallest L2
+// norm (equal norms: the lower n is pruned first); the kept columns, ascending
+// (offsetn), form tiles of G consecutive kept columns, the last one shorter;
+// tile t keeps its k_t rows k of largest L2 norm over its own columns (equal
+// norms: the lower k is kept), ascending (offsetk).  Norms are exact: every
+// fp16 value is m * 2^e with e >= -24, so w^2 * 2^48 = m^2 * 2^(2e + 48) is an
+// integer, and the sums are kept in unsigned 128-bit integers.
+// Output in the library's descriptor layout: offsetn [N - n_pruned],
+// tile_kofs [T + 1] (prefix sums of k_t rounded up to 64), offsetk
+// [tile_kofs[T]] (padded with the tile's last kept k) and Wc fp16 bits
+// [tile_kofs[T] / 64][G][64] (block b of tile t, element [j][c] = W[offsetn[t G
+// + j]][offsetk[tile_kofs[t] + 64 b + c]], +0 in unused slots).
+int orc_tw_reorganize(const uint16_t* W, int64_t N, int64_t K, int G, int64_t n_pruned, const int32_t* k_per_tile,
+                      int32_t* offsetn, int32_t* tile_kofs, int32_t* offsetk, uint16_t* Wc) {
+  typedef unsigned __int128 u128;
+  if (G != 128 || n_pruned < 0 || n_pruned >= N) return 1;
+  auto sq = [&](int64_t n, int64_t k) -> u128 {
+    const uint16_t h = W[n * K + k];
+    const int ex = (h >> 10) & 0x1F, fr = h & 0x3FF;
+    if (ex == 0x1F) return 0;  // Inf / NaN are outside the contract
+    const u128 m = ex ? u128(1024 + fr) : u128(fr);
+    const int e = ex ? ex - 25 : -24;
+    return (m * m) << (2 * e + 48);
+  };
+  // column keys and the global prune
+  std::vector<u128> ckey(static_cast<size_t>(N), 0);
+  for (int64_t n = 0; n < N; ++n)
+    for (int64_t k = 0; k < K; ++k) ckey[size_t(n)] += sq(n, k);
+  std::vector<int64_t> order(static_cast<size_t>(N));
+  for (int64_t n = 0; n < N; ++n) order[size_t(n)] = n;
+  std::sort(order.begin(), order.end(), [&](int64_t a, int64_t b) {
+    return ckey[size_t(a)] != ckey[size_t(b)] ? ckey[size_t(a)] < ckey[size_t(b)] : a < b;
+  });
+  std::vector<char> pruned(static_cast<size_t>(N), 0);
+  for (int64_t i = 0; i < n_pruned; ++i) pruned[size_t(order[size_t(i)])] = 1;
+  int64_t Nk = 0;
+  for (int64_t n = 0; n < N; ++n)
+    if (!pruned[size_t(n)]) offsetn[Nk++] = int32_t(n);
+  const int64_t T = (Nk + G - 1) / G;
+  tile_kofs[0] = 0;
+  for (int64_t t = 0; t < T; ++t) {
+    if (k_per_tile[t] < 1 || k_per_tile[t] > K) return 1;
+    tile_kofs[t + 1] = tile_kofs[t] + (k_per_tile[t] + 63) / 64 * 64;
+  }
+  std::memset(Wc, 0, size_t(tile_kofs[T]) * size_t(G) * 2);
+  // per tile: row keys over the tile's columns, top k_t rows, condensed values
+  for (int64_t t = 0; t < T; ++t) {
+    const int64_t j0 = t * G, Gt = (Nk - j0) < G ? Nk - j0 : G;
+    std::vector<u128> rkey(static_cast<size_t>(K), 0);
+    for (int64_t j = 0; j < Gt; ++j)
+      for (int64_t k = 0; k < K; ++k) rkey[size_t(k)] += sq(offsetn[j0 + j], k);
+    std::vector<int64_t> rk(static_cast<size_t>(K));
+    for (int64_t k = 0; k < K; ++k) rk[size_t(k)] = k;
+    std::sort(rk.begin(), rk.end(), [&](int64_t a, int64_t b) {
+      return rkey[size_t(a)] != rkey[size_t(b)] ? rkey[size_t(a)] > rkey[size_t(b)] : a < b;
+    });
+    const int64_t kt = k_per_tile[t];
+    std::sort(rk.begin(), rk.begin() + kt);
+    const int64_t base = tile_kofs[t];
+    for (int64_t i = 0; i < tile_kofs[t + 1] - base; ++i) offsetk[base + i] = int32_t(rk[size_t(i < kt ? i : kt - 1)]);
+    for (int64_t j = 0; j < Gt; ++j)
+      for (int64_t i = 0; i < kt; ++i) {
+        const int64_t blk = base / 64 + i / 64, c = i % 64;
+        Wc[(blk * G + j) * 64 + c] = W[int64_t(offsetn[j0 + j]) * K + rk[size_t(i)]];
+      }
+  }
   return 0;
 }
 

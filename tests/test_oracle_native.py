@@ -195,3 +195,32 @@ def test_fixed_point_epilogue_matches_numpy_bit_for_bit():
 def test_gelu_f64_matches_numpy():
     v = np.linspace(-8, 8, 4001)
     assert np.allclose(native.gelu_f64(v), s24.gelu_ref(v), rtol=1e-15, atol=1e-15)
+
+
+@pytest.mark.parametrize("seed", [0, 1])
+def test_tw_reorganize_matches_numpy_with_ties(seed):
+    """Exact-norm column prune and per-tile row selection, C++ against numpy, on
+    weights with many equal norms (values from a small set, repeated rows)."""
+    rng = np.random.default_rng(seed)
+    N, K, G = 400, 192, 128
+    W = rng.choice(np.array([0.0, 0.5, -0.5, 1.0, 2.0 ** -20, 0.25], dtype=np.float16), size=(N, K))
+    W[10] = W[11]          # equal column keys
+    W[:, 5] = W[:, 6]      # equal row keys in every tile
+    P = 37
+    T = (N - P + G - 1) // G
+    kpt = list(rng.integers(1, K + 1, T))
+    offsetn, kofs, offsetk, Wc = native.tw_reorganize(W, P, kpt)
+    r = tw.tw_reorganize(W, G, P, kpt)
+    on2, kofs2, kk2, ok2, Wc2 = native.tw_descriptor(r)
+    assert np.array_equal(offsetn, on2) and np.array_equal(kofs, kofs2)
+    assert np.array_equal(offsetk, ok2)
+    assert np.array_equal(Wc.view(np.uint16), Wc2.view(np.uint16))
+
+
+def test_tw_reorganize_bert_layer_matches_numpy():
+    d = gen.make_inputs("tw_bert_f16", layers=["attn_out"])[0]
+    offsetn, kofs, offsetk, Wc = native.tw_reorganize(d["W"], d["n_pruned"], d["k_per_tile"])
+    on2, kofs2, _kk, ok2, Wc2 = native.tw_descriptor(tw.tw_reorganize(d["W"], d["G"], d["n_pruned"],
+                                                                      d["k_per_tile"]))
+    assert np.array_equal(offsetn, on2) and np.array_equal(kofs, kofs2) and np.array_equal(offsetk, ok2)
+    assert np.array_equal(Wc.view(np.uint16), Wc2.view(np.uint16))
