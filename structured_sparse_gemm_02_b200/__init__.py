@@ -114,6 +114,48 @@ def _ptr(t) -> Optional[int]:
     return None if t is None else t.data_ptr()
 
 
+def _on_device(t, name: str) -> None:
+    """A tensor whose pointer goes to a kernel lives on the current CUDA device."""
+    import torch
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (it is on {t.device})")
+    if t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, the current device is cuda:{torch.cuda.current_device()}")
+
+
+def _arg(t, name: str, dtypes, shape=None, contiguous=False, optional=False):
+    """Check a tensor argument before its pointer reaches the library: dtype, exact
+    shape, row-major layout with unit column stride (the C ABI passes only the
+    row pitch), contiguity where the ABI fixes the pitch, and the device.
+    Returns t (None is accepted only for optional arguments)."""
+    import torch
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected one of {tuple(dtypes)}")
+    if shape is not None and tuple(t.shape) != tuple(int(v) for v in shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(int(v) for v in shape)}")
+    if t.dim() == 2 and t.numel() > 0 and t.shape[1] > 1 and t.stride(1) != 1:
+        raise ValueError(f"{name} must be row-major with unit column stride (got strides {t.stride()})")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    _on_device(t, name)
+    return t
+
+
+def _nbytes(t) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+def _types(*names):
+    import torch
+    return tuple(getattr(torch, n) for n in names)
+
+
 def version() -> int:
     return lib().spg_version()
 
@@ -136,9 +178,11 @@ def selftest_bounded_wait(limit_ns: int = 20_000_000, stream=None) -> None:
 def sparse_prune_24(W, Wm=None, stream=None):
     """2:4 magnitude prune of W [N, K] (row pitch = W.stride(0)); returns Wm."""
     import torch
+    _arg(W, "W", _types("float16", "bfloat16", "int8"))
+    N, K = W.shape
     if Wm is None:
         Wm = torch.empty_like(W)
-    N, K = W.shape
+    _arg(Wm, "Wm", (W.dtype,), (N, K))
     _check("sparse_prune_24", lib().sparse_prune_24(
         _ptr(W), W.stride(0), _ptr(Wm), Wm.stride(0), N, K, _dtype_code(W), _stream(stream)))
     return Wm
@@ -147,23 +191,39 @@ def sparse_prune_24(W, Wm=None, stream=None):
 def sparse_compress_24(W, Wv=None, meta=None, stream=None):
     """2:4 compress W [N, K] into (Wv [N, K/2], meta uint8 [N, K/8])."""
     import torch
+    _arg(W, "W", _types("float16", "bfloat16", "int8"))
     N, K = W.shape
     if Wv is None:
         Wv = torch.empty((N, K // 2), dtype=W.dtype, device=W.device)
     if meta is None:
         meta = torch.empty((N, K // 8), dtype=torch.uint8, device=W.device)
+    _arg(Wv, "Wv", (W.dtype,), (N, K // 2), contiguous=True)
+    _arg(meta, "meta", _types("uint8"), (N, K // 8), contiguous=True)
     _check("sparse_compress_24", lib().sparse_compress_24(
         _ptr(W), W.stride(0), _ptr(Wv), _ptr(meta), N, K, _dtype_code(W), _stream(stream)))
     return Wv, meta
 
 
+def _check_24(X, Wv, meta, dtypes):
+    """X [M, K], Wv [N, K/2] (same dtype, contiguous), meta [N, K/8] uint8 (contiguous); returns M, K, N."""
+    _arg(X, "X", dtypes)
+    if X.dim() != 2 or Wv is None or Wv.dim() != 2:
+        raise ValueError("X and Wv must be 2-D")
+    M, K = X.shape
+    N = Wv.shape[0]
+    _arg(Wv, "Wv", (X.dtype,), (N, K // 2), contiguous=True)
+    _arg(meta, "meta", _types("uint8"), (N, K // 8), contiguous=True)
+    return M, K, N
+
+
 def spgemm_24_f16(X, Wv, meta, bias=None, Y=None, stream=None):
     """Y [M, N] = X [M, K] . decompress(Wv, meta)^T (+ bias), fp16 or bf16."""
     import torch
-    M, K = X.shape
-    N = Wv.shape[0]
+    M, K, N = _check_24(X, Wv, meta, _types("float16", "bfloat16"))
+    _arg(bias, "bias", (X.dtype,), (N,), contiguous=True, optional=True)
     if Y is None:
         Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    _arg(Y, "Y", (X.dtype,), (M, N))
     _check("spgemm_24_f16", lib().spgemm_24_f16(
         _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(bias), _ptr(Y), Y.stride(0), M, N, K,
         _dtype_code(X), _stream(stream)))
@@ -173,10 +233,11 @@ def spgemm_24_f16(X, Wv, meta, bias=None, Y=None, stream=None):
 def spgemm_24_f16_gelu(X, Wv, meta, bias=None, Y=None, stream=None):
     """Y [M, N] = GELU(X [M, K] . decompress(Wv, meta)^T (+ bias)), fp16 or bf16."""
     import torch
-    M, K = X.shape
-    N = Wv.shape[0]
+    M, K, N = _check_24(X, Wv, meta, _types("float16", "bfloat16"))
+    _arg(bias, "bias", (X.dtype,), (N,), contiguous=True, optional=True)
     if Y is None:
         Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    _arg(Y, "Y", (X.dtype,), (M, N))
     _check("spgemm_24_f16_gelu", lib().spgemm_24_f16_gelu(
         _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(bias), _ptr(Y), Y.stride(0), M, N, K,
         _dtype_code(X), _stream(stream)))
@@ -186,10 +247,11 @@ def spgemm_24_f16_gelu(X, Wv, meta, bias=None, Y=None, stream=None):
 def spgemm_24_f16_yt(X, Wv, meta, bias=None, Yt=None, stream=None):
     """Yt [N, M] = (X [M, K] . decompress(Wv, meta)^T (+ bias))^T, fp16 or bf16."""
     import torch
-    M, K = X.shape
-    N = Wv.shape[0]
+    M, K, N = _check_24(X, Wv, meta, _types("float16", "bfloat16"))
+    _arg(bias, "bias", (X.dtype,), (N,), contiguous=True, optional=True)
     if Yt is None:
         Yt = torch.empty((N, M), dtype=X.dtype, device=X.device)
+    _arg(Yt, "Yt", (X.dtype,), (N, M))
     _check("spgemm_24_f16_yt", lib().spgemm_24_f16_yt(
         _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(bias), _ptr(Yt), Yt.stride(0), M, N, K,
         _dtype_code(X), _stream(stream)))
@@ -199,11 +261,13 @@ def spgemm_24_f16_yt(X, Wv, meta, bias=None, Yt=None, stream=None):
 def spgemm_24_s8(X, Wv, meta, scale=None, bias=None, Y=None, out_mode=SPG_OUT_F16, stream=None):
     """int8 2:4 GEMM; out_mode SPG_OUT_F16 (dequantised fp16) or SPG_OUT_S32 (raw int32)."""
     import torch
-    M, K = X.shape
-    N = Wv.shape[0]
+    M, K, N = _check_24(X, Wv, meta, _types("int8"))
+    _arg(scale, "scale", _types("float32"), (N,), contiguous=True, optional=out_mode == SPG_OUT_S32)
+    _arg(bias, "bias", _types("float16"), (N,), contiguous=True, optional=True)
+    ydt = torch.int32 if out_mode == SPG_OUT_S32 else torch.float16
     if Y is None:
-        Y = torch.empty((M, N), dtype=torch.int32 if out_mode == SPG_OUT_S32 else torch.float16,
-                        device=X.device)
+        Y = torch.empty((M, N), dtype=ydt, device=X.device)
+    _arg(Y, "Y", (ydt,), (M, N))
     _check("spgemm_24_s8", lib().spgemm_24_s8(
         _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(scale), _ptr(bias), _ptr(Y), Y.stride(0),
         out_mode, M, N, K, _stream(stream)))
@@ -214,10 +278,12 @@ def spgemm_24_s8_q(X, Wv, meta, scale, bias=None, qscale=1.0, act=SPG_ACT_NONE, 
     """int8 2:4 layer whose epilogue emits int8 activations for the next int8 layer:
     Yq = clamp(rne(act(fp32(acc) * scale (+ bias)) * qscale), -127, 127)."""
     import torch
-    M, K = X.shape
-    N = Wv.shape[0]
+    M, K, N = _check_24(X, Wv, meta, _types("int8"))
+    _arg(scale, "scale", _types("float32"), (N,), contiguous=True)
+    _arg(bias, "bias", _types("float16"), (N,), contiguous=True, optional=True)
     if Yq is None:
         Yq = torch.empty((M, N), dtype=torch.int8, device=X.device)
+    _arg(Yq, "Yq", _types("int8"), (M, N))
     _check("spgemm_24_s8_q", lib().spgemm_24_s8_q(
         _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(scale), _ptr(bias), float(qscale), int(act), _ptr(Yq),
         Yq.stride(0), M, N, K, _stream(stream)))
@@ -250,13 +316,42 @@ class TwDesc:
 def tw_reorganize(W, G: int, n_pruned: int, k_per_tile: Sequence[int], workspace=None, stream=None) -> TwDesc:
     """Condense a dense fp16 W [N, K] into a tile-wise descriptor."""
     import torch
+    _arg(W, "W", _types("float16"))
     N, K = W.shape
     d = TwDesc(N, K, G, n_pruned, k_per_tile, device=W.device)
     if workspace is None:
         workspace = torch.empty(max(16, d.sizes.reorg_ws_bytes), dtype=torch.uint8, device=W.device)
+    _arg(workspace, "workspace", (workspace.dtype,), contiguous=True)
     _check("tw_reorganize", lib().tw_reorganize(_ptr(W), W.stride(0), n_pruned, d.k_host, ctypes.byref(d.c),
-                                                _ptr(workspace), workspace.numel(), _stream(stream)))
+                                                _ptr(workspace), _nbytes(workspace), _stream(stream)))
     return d
+
+
+def _check_tw_x(X, desc, x_layout, M, dtypes):
+    """X is [M, K] (SPG_X_MK) or [K, M] (SPG_X_KM) with K the descriptor's; returns M."""
+    if x_layout not in (SPG_X_MK, SPG_X_KM):
+        raise ValueError(f"x_layout must be SPG_X_MK or SPG_X_KM, not {x_layout}")
+    _arg(X, "X", dtypes)
+    if X.dim() != 2:
+        raise ValueError("X must be 2-D")
+    if M is None:
+        M = X.shape[0] if x_layout == SPG_X_MK else X.shape[1]
+    K = desc.sizes.K
+    want = (M, K) if x_layout == SPG_X_MK else (K, M)
+    if tuple(X.shape) != want:
+        raise ValueError(f"X: shape {tuple(X.shape)}, expected {want} for this layout and descriptor")
+    return int(M)
+
+
+def _workspace(workspace, need: int, device):
+    """The caller's workspace (checked against the size the call needs) or a new one."""
+    import torch
+    if workspace is None:
+        return torch.empty(need, dtype=torch.uint8, device=device) if need else None
+    _arg(workspace, "workspace", (workspace.dtype,), contiguous=True)
+    if _nbytes(workspace) < need:
+        raise ValueError(f"workspace holds {_nbytes(workspace)} bytes, the call needs {need}")
+    return workspace
 
 
 def tw_workspace_size(M: int, K: int, x_layout: int) -> int:
@@ -267,17 +362,15 @@ def spgemm_tw_f16(X, desc: TwDesc, x_layout=SPG_X_MK, Y=None, workspace=None, M:
                   stream=None):
     """Tile-wise GEMM: X [M, K] (SPG_X_MK) or [K, M] (SPG_X_KM) -> Y [M, N] fp16."""
     import torch
-    if M is None:
-        M = X.shape[0] if x_layout == SPG_X_MK else X.shape[1]
+    M = _check_tw_x(X, desc, x_layout, M, _types("float16"))
     N = desc.sizes.N
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
-    ws = tw_workspace_size(M, desc.sizes.K, x_layout)
-    if workspace is None and ws:
-        workspace = torch.empty(ws, dtype=torch.uint8, device=X.device)
+    _arg(Y, "Y", _types("float16"), (M, N))
+    workspace = _workspace(workspace, tw_workspace_size(M, desc.sizes.K, x_layout), X.device)
     _check("spgemm_tw_f16", lib().spgemm_tw_f16(
         _ptr(X), X.stride(0), x_layout, ctypes.byref(desc.c), _ptr(Y), Y.stride(0), M, _ptr(workspace),
-        ws if workspace is not None else 0, _stream(stream)))
+        _nbytes(workspace), _stream(stream)))
     return Y
 
 
@@ -285,25 +378,27 @@ def spgemm_tw_f16_yt(X, desc: TwDesc, x_layout=SPG_X_MK, Yt=None, workspace=None
                      stream=None):
     """Tile-wise GEMM writing Yt [N, M] = Y^T (the [K, M] activations of a following tile-wise layer)."""
     import torch
-    if M is None:
-        M = X.shape[0] if x_layout == SPG_X_MK else X.shape[1]
+    M = _check_tw_x(X, desc, x_layout, M, _types("float16"))
     N = desc.sizes.N
     if Yt is None:
         Yt = torch.empty((N, M), dtype=torch.float16, device=X.device)
-    ws = tw_workspace_size(M, desc.sizes.K, x_layout)
-    if workspace is None and ws:
-        workspace = torch.empty(ws, dtype=torch.uint8, device=X.device)
+    _arg(Yt, "Yt", _types("float16"), (N, M))
+    workspace = _workspace(workspace, tw_workspace_size(M, desc.sizes.K, x_layout), X.device)
     _check("spgemm_tw_f16_yt", lib().spgemm_tw_f16_yt(
         _ptr(X), X.stride(0), x_layout, ctypes.byref(desc.c), _ptr(Yt), Yt.stride(0), M, _ptr(workspace),
-        ws if workspace is not None else 0, _stream(stream)))
+        _nbytes(workspace), _stream(stream)))
     return Yt
 
 
 def tw_condense_f32(W, desc: TwDesc, Wc32=None, stream=None):
     """fp32 condensed tiles of W [N, K] (fp32) through the pattern of ``desc``."""
     import torch
+    _arg(W, "W", _types("float32"), (desc.sizes.N, desc.sizes.K))
     if Wc32 is None:
         Wc32 = torch.empty(desc.sizes.wc_elems, dtype=torch.float32, device=W.device)
+    _arg(Wc32, "Wc32", _types("float32"), contiguous=True)
+    if Wc32.numel() < desc.sizes.wc_elems:
+        raise ValueError(f"Wc32 holds {Wc32.numel()} elements, the descriptor needs {desc.sizes.wc_elems}")
     _check("tw_condense_f32", lib().tw_condense_f32(_ptr(W), W.stride(0), ctypes.byref(desc.c), _ptr(Wc32),
                                                     _stream(stream)))
     return Wc32
@@ -313,17 +408,18 @@ def spgemm_tw_f32(X, desc: TwDesc, Wc32, x_layout=SPG_X_MK, Y=None, workspace=No
                   stream=None):
     """Tile-wise GEMM in fp32 on the CUDA cores: X [M, K] or [K, M] -> Y [M, N] fp32."""
     import torch
-    if M is None:
-        M = X.shape[0] if x_layout == SPG_X_MK else X.shape[1]
+    M = _check_tw_x(X, desc, x_layout, M, _types("float32"))
     N = desc.sizes.N
+    _arg(Wc32, "Wc32", _types("float32"), contiguous=True)
+    if Wc32.numel() < desc.sizes.wc_elems:
+        raise ValueError(f"Wc32 holds {Wc32.numel()} elements, the descriptor needs {desc.sizes.wc_elems}")
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float32, device=X.device)
-    ws = int(lib().tw_workspace_size_f32(M, desc.sizes.K, x_layout))
-    if workspace is None and ws:
-        workspace = torch.empty(ws, dtype=torch.uint8, device=X.device)
+    _arg(Y, "Y", _types("float32"), (M, N))
+    workspace = _workspace(workspace, int(lib().tw_workspace_size_f32(M, desc.sizes.K, x_layout)), X.device)
     _check("spgemm_tw_f32", lib().spgemm_tw_f32(
         _ptr(X), X.stride(0), x_layout, ctypes.byref(desc.c), _ptr(Wc32), _ptr(Y), Y.stride(0), M, _ptr(workspace),
-        ws if workspace is not None else 0, _stream(stream)))
+        _nbytes(workspace), _stream(stream)))
     return Y
 
 
@@ -335,10 +431,11 @@ def spgemm_tw_f16_noalloc(X, desc: TwDesc, Y=None, stream=None):
     overlap on the GPU.
     """
     import torch
-    M = X.shape[0]
+    M = _check_tw_x(X, desc, SPG_X_MK, None, _types("float16"))
     N = desc.sizes.N
     if Y is None:
         Y = torch.empty((M, N), dtype=torch.float16, device=X.device)
+    _arg(Y, "Y", _types("float16"), (M, N))
     _check("spgemm_tw_f16_noalloc", lib().spgemm_tw_f16_noalloc(
         _ptr(X), X.stride(0), ctypes.byref(desc.c), _ptr(Y), Y.stride(0), M, _stream(stream)))
     return Y
