@@ -49,6 +49,16 @@ def test_host_only_calls():
     assert sz.reorg_ws_bytes >= 768 * 20
     assert L.tw_query_sizes(768, 768, 64, 77, kpt, ctypes.byref(sz)) == 2      # G must be 128
     assert L.tw_query_sizes(768, 768, 128, 768, kpt, ctypes.byref(sz)) == 1    # n_pruned < N
+    one = (ctypes.c_int32 * 1)(768)
+    assert L.tw_query_sizes(768, 768, 128, 767, one, ctypes.byref(sz)) == 0    # one kept column, all K rows
+    assert (sz.Nk, sz.T, sz.offsetk_len) == (1, 1, 768)
+    bad = (ctypes.c_int32 * 6)(260, 0, 272, 118, 245, 187)
+    assert L.tw_query_sizes(768, 768, 128, 77, bad, ctypes.byref(sz)) == 1     # a tile keeping no row
+    bad[1] = 769
+    assert L.tw_query_sizes(768, 768, 128, 77, bad, ctypes.byref(sz)) == 1     # k_t > K
+    assert L.tw_query_sizes(768, 760, 128, 77, kpt, ctypes.byref(sz)) == 2     # K % 64
+    assert L.tw_query_sizes(768, 8256, 128, 77, kpt, ctypes.byref(sz)) == 2    # K above the reorganiser's limit
+    assert L.tw_query_sizes(768, 768, 128, 77, None, ctypes.byref(sz)) == 1
     assert L.tw_workspace_size(4096, 768, spg.SPG_X_MK) == 4096 * 768 * 2
     assert L.tw_workspace_size(4096, 768, spg.SPG_X_KM) == 0
 
