@@ -224,3 +224,23 @@ def test_tw_reorganize_bert_layer_matches_numpy():
                                                                       d["k_per_tile"]))
     assert np.array_equal(offsetn, on2) and np.array_equal(kofs, kofs2) and np.array_equal(offsetk, ok2)
     assert np.array_equal(Wc.view(np.uint16), Wc2.view(np.uint16))
+
+
+def test_tw_reorganize_figure_spans_golden():
+    """The C++ reorganisation reproduces the tile spans of the "Re-organize"
+    figure (G + 4, G + 3, G + 2, G - 9; tests/golden/tw_reorganize_figure.txt)."""
+    spec = {}
+    with open(os.path.join(GOLDEN, "tw_reorganize_figure.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                tag, *rest = line.split()
+                spec[tag] = [int(v) for v in rest]
+    G, N, K = spec["G"][0], spec["N"][0], spec["K"][0]
+    W = np.full((N, K), 1.0, dtype=np.float16)
+    W[spec["PRUNED"], :] = np.float16(0.001)
+    offsetn, kofs, offsetk, Wc = native.tw_reorganize(W, len(spec["PRUNED"]), [K] * 4, G=G)
+    assert sorted(set(range(N)) - set(offsetn.tolist())) == spec["PRUNED"]
+    starts = [0] + [int(offsetn[t * G]) for t in range(1, 4)] + [N]
+    assert [starts[t + 1] - starts[t] for t in range(4)] == spec["SPANS"]
+    assert [min(G, len(offsetn) - t * G) for t in range(4)] == spec["KEPT_PER_TILE"]
