@@ -150,3 +150,38 @@ def test_empty_batch_is_a_no_op():
     assert L.spgemm_tw_f16(None, 768, spg.SPG_X_MK, d, None, 700, 0, None, 0, None) == 1      # ldy < N
     # the entry point without allocation keeps M >= 8 (its limits are its own)
     assert L.spgemm_tw_f16_noalloc(None, 768, d, None, 768, 0, None) == 1
+
+
+def test_plain_c_program_uses_the_abi(tmp_path):
+    """The header is valid C99 and every declared entry point links with C
+    linkage: a C program takes the address of each one, links against the
+    library and runs the host-only calls."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("gcc not available")
+    import structured_sparse_gemm_02_b200 as spg
+    spg.lib()
+    names = sorted(_declared())
+    src = tmp_path / "use_abi.c"
+    src.write_text(
+        "#include <stdio.h>\n#include \"spgemm.h\"\n"
+        "int main(void) {\n"
+        "  void* fns[] = {" + ", ".join(f"(void*){n}" for n in names) + "};\n"
+        "  int32_t kpt[6] = {260, 290, 272, 118, 245, 187};\n"
+        "  spg_tw_sizes sz;\n"
+        "  spg_status st = tw_query_sizes(768, 768, 128, 77, kpt, &sz);\n"
+        "  for (unsigned i = 0; i < sizeof(fns) / sizeof(fns[0]); ++i) if (!fns[i]) return 2;\n"
+        "  printf(\"%d %d %lld %d %s\\n\", spg_version(), (int)st, (long long)sz.Nk, sz.T,\n"
+        "         spg_status_string(SPG_ERR_TIMEOUT));\n"
+        "  return 0;\n}\n")
+    libdir = os.path.dirname(spg.LIB_PATH)
+    exe = tmp_path / "use_abi"
+    p = subprocess.run([gcc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"), str(src),
+                        "-L", libdir, "-lspgemm", f"-Wl,-rpath,{libdir}", "-o", str(exe)],
+                       capture_output=True, text=True)
+    assert p.returncode == 0, p.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.split() == ["10000", "0", "691", "6", "SPG_ERR_TIMEOUT"]
