@@ -244,3 +244,31 @@ def test_tw_reorganize_figure_spans_golden():
     starts = [0] + [int(offsetn[t * G]) for t in range(1, 4)] + [N]
     assert [starts[t + 1] - starts[t] for t in range(4)] == spec["SPANS"]
     assert [min(G, len(offsetn) - t * G) for t in range(4)] == spec["KEPT_PER_TILE"]
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=40, deadline=None)
+@given(N=st.integers(1, 24), G8=st.integers(1, 12), dtype=st.sampled_from(["f16", "bf16", "s8"]),
+       alphabet=st.integers(2, 9), seed=st.integers(0, 2 ** 31 - 1))
+def test_property_two_oracles_agree_on_2to4(N, G8, dtype, alphabet, seed):
+    """Random shapes and values drawn from a small alphabet (so that equal
+    magnitudes are common): both oracles select, store and, for int8, multiply
+    identically."""
+    rng = np.random.default_rng(seed)
+    K = 8 * G8
+    vals = rng.integers(-alphabet, alphabet + 1, (N, K))
+    if dtype == "s8":
+        W = vals.astype(np.int8)
+    elif dtype == "f16":
+        W = (vals * 0.125).astype(np.float16)
+    else:
+        W = gen.f32_to_bf16_bits((vals * 0.125).astype(np.float32))
+    Wv, meta = native.compress_24(W, dtype)
+    Wv2, meta2 = s24.compress_24(W, dtype)
+    assert np.array_equal(meta, meta2)
+    assert np.array_equal(Wv.view(np.uint8), np.ascontiguousarray(Wv2).view(np.uint8))
+    if dtype == "s8":
+        X = rng.integers(-127, 128, (5, K)).astype(np.int8)
+        assert np.array_equal(native.gemm_24_s8_ref(X, Wv, meta), s24.gemm_24_s8_ref(X, Wv, meta))
