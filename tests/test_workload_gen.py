@@ -69,3 +69,40 @@ def test_int8_weight_recipe():
     # every row reaches +-127 exactly once its max is divided by its own scale
     assert (np.abs(q.astype(np.int32)).max(axis=1) == 127).all()
     assert s.dtype == np.float32 and (s > 0).all()
+
+
+def _quant_golden():
+    import os
+    path = os.path.join(os.path.dirname(__file__), "golden", "int8_weight_quant.txt")
+    rows, scales, codes = [], [], []
+    for line in open(path):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        tag, *vals = line.split()
+        if tag == "w":
+            rows.append([float(v) for v in vals])
+        elif tag == "s":
+            scales.append(int(vals[0], 16))
+        elif tag == "q":
+            codes.append([int(v) for v in vals])
+    return (np.array(rows, dtype=np.float32), np.array(scales, dtype=np.uint32), np.array(codes, dtype=np.int8))
+
+
+def test_int8_weight_quantisation_hand_worked_golden():
+    """The per-row scale and the codes of a few hand-worked rows, ties to even
+    included (tests/golden/int8_weight_quant.txt)."""
+    w, s_bits, q_want = _quant_golden()
+    assert w.shape == (4, 8)
+    q, s = gen.quantize_weight_s8(w)
+    assert q.dtype == np.int8 and s.dtype == np.float32
+    assert np.array_equal(s.view(np.uint32), s_bits)
+    assert np.array_equal(q, q_want)
+
+
+def test_int8_weight_recipe_is_the_workload_step():
+    """The int8 ViT-L workload's weights are quantize_weight_s8 of its fp32 draws."""
+    d = gen.make_inputs("vitl_mlp_s8")[0]
+    w = gen.normal(0, "vitl_mlp_s8.fc1.W", 4 * 1024, 0.02).reshape(4, 1024)
+    q, s = gen.quantize_weight_s8(w)
+    assert np.array_equal(d["W"][:4], q) and np.array_equal(d["scale"][:4], s)

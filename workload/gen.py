@@ -175,6 +175,24 @@ CONFIGS: Dict[str, Config] = {
 }
 
 
+def quantize_weight_s8(w: np.ndarray):
+    """Symmetric per-row int8 weights of the int8 ViT-Large workload.
+
+    Per row n, in fp32: ``s[n] = max_k |w[n, k]| / 127`` (one fp32 division,
+    round to nearest even; an all-zero row takes s = 1), then
+    ``q = clamp(rne(w / s[n]), -127, 127)`` with the division in fp32 and ties
+    rounded to even.  Returns ``(q int8 [N, K], s float32 [N])``.  ("Boost
+    Vision Transformer with GPU-Friendly Sparsity and Quantization",
+    Abstract: the 2:4 model quantised to integer tensors; the rounding mode
+    is not stated there, round-to-nearest-even is the reading.)  The 2:4
+    selection on |q| happens afterwards, in the method."""
+    w = np.asarray(w, dtype=np.float32)
+    s = (np.abs(w).max(axis=1) / np.float32(127.0)).astype(np.float32)
+    s = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
+    q = np.clip(np.rint((w / s[:, None]).astype(np.float32)), -127, 127).astype(np.int8)
+    return q, s
+
+
 def tw_tile_counts(N: int, G: int, frac: float):
     """(P, Nk, T): pruned columns round-half-even(frac*N), kept columns, tiles of G kept columns."""
     P = int(np.rint(frac * N))
@@ -193,9 +211,7 @@ def _layer_inputs(cfg: Config, seed: int, lname: str, M: int, N: int, K: int, bi
     if cfg.kind == "24_s8":
         d["X"] = uniform_int127(seed, xstem, M * K).reshape(M, K)
         w = normal(seed, wstem + ".W", N * K, cfg.w_std).reshape(N, K)
-        s = (np.abs(w).max(axis=1) / np.float32(127.0)).astype(np.float32)
-        s = np.where(s > 0, s, np.float32(1.0)).astype(np.float32)
-        q = np.clip(np.rint(w / s[:, None]), -127, 127).astype(np.int8)
+        q, s = quantize_weight_s8(w)
         d["W"] = q
         d["scale"] = s
         d["bias"] = f32_to_f16(normal(seed, stem + ".bias", N, cfg.bias_std)) if bias else None
