@@ -27,6 +27,11 @@
  *    that word.
  *  - Device requirement: compute capability 10.0 (B200, sm_100a); other
  *    devices get SPG_ERR_UNSUPPORTED_DEVICE.
+ *  - The library looks up the device addresses of its own device arrays (the
+ *    error word, the scratch of spgemm_tw_f16_noalloc) once per device and
+ *    keeps them for the life of the process.  Do not use it across
+ *    cudaDeviceReset() or any other teardown of a device's primary context:
+ *    the kept addresses would no longer be valid.
  *  - An empty batch (M == 0) is valid for every GEMM entry point except
  *    spgemm_tw_f16_noalloc: the other arguments are validated as usual,
  *    nothing is launched, SPG_OK is returned, and X, Y (and the workspace)
@@ -66,10 +71,13 @@ int spg_version(void);
 /* Static, human-readable name of a status code. */
 const char* spg_status_string(spg_status s);
 
-/* Synchronises `stream`, then reads and clears the current device's error
- * word.  Returns SPG_ERR_TIMEOUT if any kernel gave up on a bounded wait since
- * the last check (the bits are stored in *bits if bits != NULL),
- * SPG_ERR_CUDA if the synchronisation failed, SPG_OK otherwise. */
+/* Takes the current device's error word and clears it in one atomic step
+ * (a one-thread kernel on `stream`), synchronises `stream` and returns what
+ * it took.  Returns SPG_ERR_TIMEOUT if any kernel gave up on a bounded wait
+ * since the last check (the bits are stored in *bits if bits != NULL),
+ * SPG_ERR_CUDA if the launch or the synchronisation failed, SPG_OK
+ * otherwise.  A bit set by a kernel still running on another stream is
+ * either taken by this call or left for the next one, never lost. */
 spg_status spg_check_device_error(spg_stream_t stream, uint32_t* bits);
 
 /* Self-test of the failure path every kernel uses (no counterpart on the
@@ -127,9 +135,11 @@ spg_status sparse_compress_24(const void* W, int64_t ldw, void* Wv, uint8_t* met
  *   Wv, meta: as written by sparse_compress_24 for [N, K]
  *   bias [N] or NULL
  *   Y    [M, N], pitch ldy >= N
- * Limits: K % 128 == 0, K >= 128; M >= 0, N >= 1 (any value, ragged tiles are
+ * Limits: K % 64 == 0, K >= 64; M >= 0, N >= 1 (any value, ragged tiles are
  * handled); M, N, K < 2^31.  X, Wv, Y 16-byte aligned; ldx and ldy in bytes
- * multiples of 16; meta 16-byte aligned; bias 2-byte aligned.
+ * multiples of 16; meta 16-byte aligned; bias 2-byte aligned.  (K % 128 != 0
+ * is served by a last pipeline stage of half depth; its metadata rows of K/8
+ * bytes are then read without TMA.)
  * ------------------------------------------------------------------------- */
 spg_status spgemm_24_f16(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,
                          void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, spg_dtype dtype,
@@ -176,7 +186,7 @@ spg_status spgemm_24_f16_yt(const void* X, int64_t ldx, const void* Wv, const ui
  *   X int8 [M, K] pitch ldx; Wv int8 [N, K/2] + meta [N, K/8] from
  *   sparse_compress_24 (dtype SPG_S8); scale fp32 [N] (required for F16,
  *   ignored for S32); bias fp16 [N] or NULL; Y [M, N] pitch ldy.
- * Limits: K % 256 == 0, K >= 256; |acc| must fit int32 (K <= 2^17 is always
+ * Limits: K % 128 == 0, K >= 128; |acc| must fit int32 (K <= 2^17 is always
  * safe); same alignment rules as spgemm_24_f16 (ldy in bytes a multiple of
  * 16); scale 4-byte aligned.
  * ------------------------------------------------------------------------- */
@@ -276,8 +286,9 @@ spg_status tw_query_sizes(int64_t N, int64_t K, int32_t G, int64_t n_pruned, con
 spg_status tw_reorganize(const void* W, int64_t ldw, int64_t n_pruned, const int32_t* k_per_tile,
                          const spg_tw_desc* desc, void* workspace, size_t ws_bytes, spg_stream_t stream);
 
-/* Workspace bytes spgemm_tw_f16 needs: M*K*2 (rounded up to 256) for
- * x_layout SPG_X_MK (the transposed activations), 0 for SPG_X_KM. */
+/* Workspace bytes spgemm_tw_f16 needs: K*M8*2 with M8 = M rounded up to a
+ * multiple of 8 (rounded up to 256 bytes) for x_layout SPG_X_MK (the
+ * transposed activations, rows padded to 16 bytes), 0 for SPG_X_KM. */
 size_t tw_workspace_size(int64_t M, int64_t K, int x_layout);
 
 /* Y = X . Wd^T with Wd the tile-wise weight described by `desc` [TW,
@@ -287,9 +298,11 @@ size_t tw_workspace_size(int64_t M, int64_t K, int x_layout);
  * [K, M] pitch ldx (SPG_X_KM: the transpose is assumed fused upstream).  Y
  * fp16 [M, N] pitch ldy; every element of Y is written (pruned columns +0).
  * fp32 accumulation, one round-to-nearest-even.
- * Limits: M % 8 == 0 (the [K, M] rows are TMA rows), M >= 0; X and
- * workspace 16-byte aligned, ldx a multiple of 8; Y 2-byte aligned, any
- * ldy >= N; ws_bytes >= tw_workspace_size(M, K, x_layout). */
+ * Limits: any M >= 0 (M < 2^31; a ragged last block of rows is handled);
+ * X and workspace 16-byte aligned, ldx a multiple of 8 (for SPG_X_KM with
+ * M % 8 != 0 the caller pads the rows of X to a multiple of 8 elements);
+ * Y 2-byte aligned, any ldy >= N; ws_bytes >= tw_workspace_size(M, K,
+ * x_layout). */
 spg_status spgemm_tw_f16(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Y,
                          int64_t ldy, int64_t M, void* workspace, size_t ws_bytes, spg_stream_t stream);
 
@@ -340,8 +353,9 @@ spg_status spgemm_tw_f32(const float* X, int64_t ldx, int x_layout, const spg_tw
  * kept in a fixed 8 MiB device array inside the library instead of a
  * caller-provided workspace; the caller still passes X, the descriptor and Y.
  *   Same arguments, limits and results as spgemm_tw_f16(X, ldx, SPG_X_MK, desc,
- *   Y, ldy, M, ...), and additionally M * K * 2 <= 8 MiB, else
- *   SPG_ERR_UNSUPPORTED_SHAPE (nothing is launched).
+ *   Y, ldy, M, ...), and additionally K * M8 * 2 <= 8 MiB with M8 = M rounded
+ *   up to a multiple of 8, else SPG_ERR_UNSUPPORTED_SHAPE (nothing is
+ *   launched).
  *   The array is allocated when the library is loaded and every GPU that
  *   loads it holds the 8 MiB until the process exits.  No call allocates or
  *   frees memory.  The first call on a device looks up the array's device

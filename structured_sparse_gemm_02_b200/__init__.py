@@ -380,8 +380,8 @@ def spgemm_tw_f16_yt(X, desc: TwDesc, x_layout=SPG_X_MK, Yt=None, workspace=None
     import torch
     M = _check_tw_x(X, desc, x_layout, M, _types("float16"))
     N = desc.sizes.N
-    if Yt is None:
-        Yt = torch.empty((N, M), dtype=torch.float16, device=X.device)
+    if Yt is None:  # rows of Yt padded to a multiple of 8 elements (the ABI's 16-byte pitch)
+        Yt = torch.empty((N, (M + 7) // 8 * 8), dtype=torch.float16, device=X.device)[:, :M]
     _arg(Yt, "Yt", _types("float16"), (N, M))
     workspace = _workspace(workspace, tw_workspace_size(M, desc.sizes.K, x_layout), X.device)
     _check("spgemm_tw_f16_yt", lib().spgemm_tw_f16_yt(

@@ -15,7 +15,12 @@
 //              order the tensor cores read it (permute_meta_f16), then
 //              arrives on the leader's barrier of the stage, which completes
 //              once both CTAs' operands have landed and both metadata warps
-//              have arrived
+//              have arrived.  When K % 128 != 0 the canonical metadata rows
+//              (K/8 bytes) are not 16-byte multiples, which a TMA map needs:
+//              this warp then reads them from global memory itself.
+// K is a multiple of the MMA pair of a stage (64 for fp16/bf16, 128 for
+// int8): a last stage with half the K of the others issues two MMAs instead
+// of four, and its out-of-range operand columns are zero-filled by TMA.
 //   warp 2     TMEM owner and MMA issuer (one thread of the leader CTA):
 //              waits for a stage, then issues it (tcgen05.cp of the
 //              metadata into tensor memory, tcgen05.mma.sp into one of two
@@ -190,6 +195,49 @@ __device__ __forceinline__ void permute_meta_f16(const uint8_t* stg, uint8_t* ou
   }
 }
 
+// The same arrangement read straight from the canonical metadata in global
+// memory (rows of `pitch` bytes, 8-byte aligned): 16 bytes of rows n0 + r,
+// starting at byte col0, of which `valid` (8 or 16) are inside the row; rows
+// at or past N and bytes past `valid` read as zero.
+__device__ __forceinline__ uint4 load_meta_row16(const uint8_t* meta, int64_t pitch, int row, int N, int col0,
+                                                 int valid) {
+  uint4 v = make_uint4(0u, 0u, 0u, 0u);
+  if (row < N) {
+    const uint2* src = reinterpret_cast<const uint2*>(meta + int64_t(row) * pitch + col0);
+    const uint2 lo = __ldg(src);
+    v.x = lo.x;
+    v.y = lo.y;
+    if (valid > 8) {
+      const uint2 hi = __ldg(src + 1);
+      v.z = hi.x;
+      v.w = hi.y;
+    }
+  }
+  return v;
+}
+
+__device__ __forceinline__ void permute_meta_f16_direct(const uint8_t* meta, int64_t pitch, int n0, int N, int col0,
+                                                        int valid, uint8_t* out, int lane) {
+#pragma unroll
+  for (int pp = 0; pp < 2; ++pp) {
+    const int p = lane + 32 * pp;
+    const int r = (p & 7) + 16 * (p >> 3);
+    const uint4 a = load_meta_row16(meta, pitch, n0 + r, N, col0, valid);
+    const uint4 b = load_meta_row16(meta, pitch, n0 + r + 8, N, col0, valid);
+    uint4 lo, hi;
+    lo.x = __byte_perm(a.x, b.x, 0x5410);
+    lo.y = __byte_perm(a.y, b.y, 0x5410);
+    lo.z = __byte_perm(a.z, b.z, 0x5410);
+    lo.w = __byte_perm(a.w, b.w, 0x5410);
+    hi.x = __byte_perm(a.x, b.x, 0x7632);
+    hi.y = __byte_perm(a.y, b.y, 0x7632);
+    hi.z = __byte_perm(a.z, b.z, 0x7632);
+    hi.w = __byte_perm(a.w, b.w, 0x7632);
+    *reinterpret_cast<uint4*>(out + r * 16) = lo;
+    *reinterpret_cast<uint4*>(out + (r + 8) * 16) = hi;
+  }
+}
+
 // Wait used only while tearing down: ignores the abort flag, still bounded.
 __device__ __forceinline__ void tail_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
   int never = 0;
@@ -300,7 +348,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
                     const __grid_constant__ CUtensorMap tmE, const __grid_constant__ CUtensorMap tmY,
                     void* __restrict__ Yp, int64_t ldy, const void* __restrict__ bias,
                     const float* __restrict__ scale, float qscale, int M, int N, int K, int band,
-                    uint32_t* err) {
+                    const uint8_t* __restrict__ meta_g, int meta_direct, uint32_t* err) {
   using C = Cfg<kInt8, BN, OUT>;
   constexpr int STAGES = C::STAGES;
   constexpr int BNH = C::BNH;
@@ -319,7 +367,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   const uint32_t rank = cluster_ctarank();
   const bool leader = rank == 0;
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
-  const int KB = K / C::KSTEP;
+  const int KB = (K + C::KSTEP - 1) / C::KSTEP;
+  // MMAs of the last stage: 4, or 2 when K ends half-way through a stage
+  const int last_mmas = (K % C::KSTEP) ? 2 : 4;
   const int NT = (N + 255) / 256;
   const int MT = (M + BN - 1) / BN;
   const int total = NT * MT;
@@ -389,7 +439,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           if constexpr (kInt8) {
             tma_load_2d_pair(e_s, &tmE, kb * 32, n0, fb);
             tma_load_2d_pair(e_s + 2048, &tmE, kb * 32 + 16, n0, fb);
-          } else {
+          } else if (!meta_direct) {
             mbar_arrive_expect_tx(&mtma[s], C::MSTG_BYTES);
             tma_load_2d(e_s, &tmE, kb * 16, n0, &mtma[s]);
           }
@@ -400,7 +450,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       // metadata barriers this CTA's metadata.
       for (uint32_t q = (g > uint32_t(STAGES) ? g - STAGES : 0u); q < g; ++q) {
         if (leader) tail_wait(&full[q % STAGES], (q / STAGES) & 1, err);
-        if constexpr (!kInt8) tail_wait(&mtma[q % STAGES], (q / STAGES) & 1, err);
+        if constexpr (!kInt8)
+          if (!meta_direct) tail_wait(&mtma[q % STAGES], (q / STAGES) & 1, err);
       }
     }
   } else if (warp == 1) {
@@ -408,14 +459,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     if constexpr (!kInt8) {
       uint32_t g = 0;
       bool ok = true;
+      const int64_t mpitch = K / 8;
       for (int t = pair; ok && t < total; t += npairs) {
+        int nt, mt;
+        tile_coords(t, NT, MT, band, nt, mt);
+        const int n0 = nt * 256 + 128 * int(rank);
         for (int kb = 0; kb < KB; ++kb, ++g) {
           const int s = g % STAGES;
-          if (!mbar_wait_warp(&mtma[s], (g / STAGES) & 1, abort_flag, err, ERR_WAIT_META)) {
-            ok = false;
-            break;
+          if (meta_direct) {
+            // the stage's previous MMAs (and their tcgen05.cp of this slot) are done
+            const uint32_t use = g / STAGES;
+            if (use > 0 && !mbar_wait_warp(&empty[s], (use - 1) & 1, abort_flag, err, ERR_WAIT_META)) {
+              ok = false;
+              break;
+            }
+            const int col0 = kb * 16;
+            permute_meta_f16_direct(meta_g, mpitch, n0, N, col0, int(mpitch) - col0 >= 16 ? 16 : 8,
+                                    smem + C::OFF_MCP + s * C::MCP_BYTES, lane);
+          } else {
+            if (!mbar_wait_warp(&mtma[s], (g / STAGES) & 1, abort_flag, err, ERR_WAIT_META)) {
+              ok = false;
+              break;
+            }
+            permute_meta_f16(smem + C::OFF_MSTG + s * C::MSTG_BYTES, smem + C::OFF_MCP + s * C::MCP_BYTES, lane);
           }
-          permute_meta_f16(smem + C::OFF_MSTG + s * C::MSTG_BYTES, smem + C::OFF_MCP + s * C::MCP_BYTES, lane);
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) mbar_arrive_cluster(full_l + 8u * s);
@@ -475,8 +542,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
             const uint32_t ecol = tmem + C::META_COL + (g & 1) * C::MCOLS;
             tc_cp_128x128b_pair(ecol, ed);
             if constexpr (kInt8) tc_cp_128x128b_pair(ecol + 4, ed + (2048 >> 4));
+            const int nmma = kb + r + 1 == KB ? last_mmas : 4;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
+              if (j >= nmma) break;
               const uint64_t adesc = ad + uint64_t((32 * j) >> 4);
               const uint64_t bdesc = bd + uint64_t(((j >> 1) * (BNH * 128) + (j & 1) * 64) >> 4);
               const uint32_t e = kInt8 ? ecol + 2 * j : ecol + (j & ~1);
@@ -730,11 +799,19 @@ spg_status launch(const void* X, int64_t ldx, const void* Wv, const uint8_t* met
                   float qscale) {
   using C = Cfg<kInt8, BN, OUT>;
   const int es = kInt8 ? 1 : 2;
+  // metadata rows of K/8 bytes: a TMA map needs a pitch that is a multiple of
+  // 16 bytes (K % 128 == 0); otherwise the metadata warp reads them directly
+  // (fp16/bf16 only: int8 K is a multiple of 128)
+  const int meta_direct = (K / 8) % 16 != 0 ? 1 : 0;
   CUtensorMap tmA, tmB, tmE, tmY;
   if (!make_tmap_2d(&tmA, Wv, es, uint64_t(K / 2), uint64_t(N), uint64_t(K / 2) * es, 128 / es, 128, true) ||
-      !make_tmap_2d(&tmB, X, es, uint64_t(K), uint64_t(M), uint64_t(ldx) * es, 128 / es, C::BNH, true) ||
-      !make_tmap_2d(&tmE, meta, 1, uint64_t(K / 8), uint64_t(N), uint64_t(K / 8), 16, 128, false))
+      !make_tmap_2d(&tmB, X, es, uint64_t(K), uint64_t(M), uint64_t(ldx) * es, 128 / es, C::BNH, true))
     return SPG_ERR_CUDA;
+  if (meta_direct)
+    std::memset(&tmE, 0, sizeof(tmE));
+  else if (!make_tmap_2d(&tmE, meta, 1, uint64_t(K / 8), uint64_t(N), uint64_t(K / 8), 16, 128, false))
+    return SPG_ERR_CUDA;
+  if (kInt8 && meta_direct) return SPG_ERR_UNSUPPORTED_SHAPE;
   // the output map: Y^T boxes [32 n][32 m] with 64-byte swizzle, Y boxes of 64
   // (16-bit) or 32 (32-bit) columns x 32 rows; int8 outputs are stored without TMA
   bool ymap_ok = true;
@@ -767,7 +844,7 @@ spg_status launch(const void* X, int64_t ldx, const void* Wv, const uint8_t* met
   band = (nt_all + nbands - 1) / nbands;  // equal bands (64 tiles: 4 x 16, not 3 x 21 + 1)
   if (launch_pdl(kern, dim3(2 * pairs), dim3(C::THREADS), C::SMEM, stream, tmA, tmB, tmE, tmY, Y, ldy, bias, scale,
                  qscale, static_cast<int>(M), static_cast<int>(N), static_cast<int>(K), static_cast<int>(band),
-                 err) != cudaSuccess)
+                 meta, meta_direct, err) != cudaSuccess)
     return SPG_ERR_CUDA;
   return launch_status();
 }
@@ -825,7 +902,7 @@ spg_status spgemm_24_f16(const void* X, int64_t ldx, const void* Wv, const uint8
   using namespace spg;
   using namespace spg::gemm24;
   if (dtype != SPG_F16 && dtype != SPG_BF16) return SPG_ERR_INVALID_ARG;
-  spg_status st = validate_common(X, ldx, Wv, meta, Y, ldy, M, N, K, 2, 2, 128);
+  spg_status st = validate_common(X, ldx, Wv, meta, Y, ldy, M, N, K, 2, 2, 64);
   if (st != SPG_OK) return st;
   if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;
   if (M == 0) return SPG_OK;  // empty batch: nothing to compute
@@ -842,7 +919,7 @@ spg_status spgemm_24_f16_gelu(const void* X, int64_t ldx, const void* Wv, const 
   using namespace spg;
   using namespace spg::gemm24;
   if (dtype != SPG_F16 && dtype != SPG_BF16) return SPG_ERR_INVALID_ARG;
-  spg_status st = validate_common(X, ldx, Wv, meta, Y, ldy, M, N, K, 2, 2, 128);
+  spg_status st = validate_common(X, ldx, Wv, meta, Y, ldy, M, N, K, 2, 2, 64);
   if (st != SPG_OK) return st;
   if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;
   if (M == 0) return SPG_OK;  // empty batch: nothing to compute
@@ -860,7 +937,7 @@ spg_status spgemm_24_f16_yt(const void* X, int64_t ldx, const void* Wv, const ui
   using namespace spg;
   using namespace spg::gemm24;
   if (dtype != SPG_F16 && dtype != SPG_BF16) return SPG_ERR_INVALID_ARG;
-  spg_status st = validate_common(X, ldx, Wv, meta, Yt, ldyt, M, N, K, 2, 2, 128, true);
+  spg_status st = validate_common(X, ldx, Wv, meta, Yt, ldyt, M, N, K, 2, 2, 64, true);
   if (st != SPG_OK) return st;
   if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;
   if (M == 0) return SPG_OK;  // empty batch: nothing to compute
@@ -879,7 +956,7 @@ spg_status spgemm_24_s8(const int8_t* X, int64_t ldx, const int8_t* Wv, const ui
   using namespace spg::gemm24;
   if (out_mode != SPG_OUT_F16 && out_mode != SPG_OUT_S32) return SPG_ERR_INVALID_ARG;
   const int out_es = out_mode == SPG_OUT_S32 ? 4 : 2;
-  spg_status st = validate_common(X, ldx, Wv, meta, Y, ldy, M, N, K, 1, out_es, 256);
+  spg_status st = validate_common(X, ldx, Wv, meta, Y, ldy, M, N, K, 1, out_es, 128);
   if (st != SPG_OK) return st;
   if (out_mode == SPG_OUT_F16 && !scale) return SPG_ERR_INVALID_ARG;
   if (scale && !aligned(scale, 4)) return SPG_ERR_MISALIGNED;
@@ -902,7 +979,7 @@ spg_status spgemm_24_s8_q(const int8_t* X, int64_t ldx, const int8_t* Wv, const 
   using namespace spg::gemm24;
   if (act != SPG_ACT_NONE && act != SPG_ACT_GELU) return SPG_ERR_INVALID_ARG;
   if (!scale || !(qscale > 0.f) || !(qscale < 3.0e38f)) return SPG_ERR_INVALID_ARG;
-  spg_status st = validate_common(X, ldx, Wv, meta, Yq, ldy, M, N, K, 1, 1, 256);
+  spg_status st = validate_common(X, ldx, Wv, meta, Yq, ldy, M, N, K, 1, 1, 128);
   if (st != SPG_OK) return st;
   if (!aligned(scale, 4)) return SPG_ERR_MISALIGNED;
   if (bias && !aligned(bias, 2)) return SPG_ERR_MISALIGNED;

@@ -183,7 +183,9 @@ __global__ void gather_wc_kernel(const uint16_t* __restrict__ W, int64_t ldw, in
 
 // ---- explicit activation transpose X [M, K] -> Xt [K, M] ------------------------------------
 // One 64 (m) x 64 (k) tile per 256-thread block, 16-byte accesses on both
-// sides (M % 8 == 0, K % 64 == 0, 16-byte aligned rows).  The tile sits in
+// sides (K % 64 == 0, 16-byte aligned rows; Xt's pitch ldt is M rounded up
+// to a multiple of 8, and the columns past M in the last 8-wide chunk are
+// written as zeros).  The tile sits in
 // shared memory as 32-bit pairs (k, k+1) with a row pitch of 33 words, so
 // both the row-wise stores and the column-wise reads are free of bank
 // conflicts.  Reads: thread t takes 8 consecutive k of rows t/8 and t/8 + 32.
@@ -201,13 +203,12 @@ __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restri
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int r = (t >> 3) + 32 * h;
-      if (m0 + r < M) {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(X + int64_t(m0 + r) * ldx + k0 + 8 * c));
-        tile[r][4 * c + 0] = v.x;
-        tile[r][4 * c + 1] = v.y;
-        tile[r][4 * c + 2] = v.z;
-        tile[r][4 * c + 3] = v.w;
-      }
+      const uint4 v = m0 + r < M ? __ldg(reinterpret_cast<const uint4*>(X + int64_t(m0 + r) * ldx + k0 + 8 * c))
+                                 : make_uint4(0u, 0u, 0u, 0u);
+      tile[r][4 * c + 0] = v.x;
+      tile[r][4 * c + 1] = v.y;
+      tile[r][4 * c + 2] = v.z;
+      tile[r][4 * c + 3] = v.w;
     }
   }
   __syncthreads();
@@ -357,7 +358,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     while (ok && u < units) {
       const int mb = (u % MB) * BN;
       const int mcol = mb + 64 * a + 8 * c;
-      const uint32_t src_bytes = mcol < M ? 16u : 0u;
+      // the chunk of 8 m at mcol: whole, cut at M (the rest zero-filled), or empty
+      const uint32_t src_bytes = mcol + 8 <= M ? 16u : mcol < M ? uint32_t(2 * (M - mcol)) : 0u;
       const uint16_t* xcol = xt + (src_bytes ? mcol : 0);
       // scalars of the next unit, loaded while this one is issued
       const int un = u + gridDim.x;
@@ -503,7 +505,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         // Y^T [N][M]: this lane's kept column nj is row nj of Y^T, and its 64
         // rows m are 128 contiguous bytes of that row, stored from registers;
         // the pruned columns it owns (its gap, and the tile's lead for j = 0)
-        // are rows of zeros.  rows is a multiple of 8 (M % 8 == 0).
+        // are rows of zeros.  Yt's pitch is a multiple of 8 elements, so
+        // whole 8-row chunks are 16-byte stores; a ragged end (M % 8) is
+        // written element by element.
         if (valid && rows > 0) {
           uint16_t* yrow = Y + int64_t(nj) * ldy + mb;
 #pragma unroll
@@ -519,14 +523,22 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
               for (int p = 0; p < 4; ++p) d4[p] = make_uint4(w[4 * p], w[4 * p + 1], w[4 * p + 2], w[4 * p + 3]);
             } else if (32 * cc < rows) {
+              const int left = rows - 32 * cc;  // 1..31 rows of this half
               uint4* d4 = reinterpret_cast<uint4*>(yrow + 32 * cc);
-              for (int p = 0; p < (rows - 32 * cc) / 8; ++p) d4[p] = make_uint4(w[4 * p], w[4 * p + 1], w[4 * p + 2], w[4 * p + 3]);
+#pragma unroll
+              for (int p = 0; p < 4; ++p)
+                if (8 * p + 8 <= left) d4[p] = make_uint4(w[4 * p], w[4 * p + 1], w[4 * p + 2], w[4 * p + 3]);
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (e >= (left & ~7) && e < left)
+                  yrow[32 * cc + e] = static_cast<uint16_t>((e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu));
             }
           }
           const int gap_end = j + 1 < Gt ? offsetn[j0 + j + 1] : n1;
           auto zero_row = [&](int z) {
             uint4* d4 = reinterpret_cast<uint4*>(Y + int64_t(z) * ldy + mb);
             for (int e = 0; e < rows / 8; ++e) d4[e] = make_uint4(0u, 0u, 0u, 0u);
+            for (int e = rows & ~7; e < rows; ++e) Y[int64_t(z) * ldy + mb + e] = 0;
           };
           for (int z = nj + 1; z < gap_end; ++z) zero_row(z);
           if (j == 0)
@@ -689,6 +701,11 @@ spg_status launch_gemm(const uint16_t* xt, int64_t ldt, const spg_tw_desc* desc,
   return launch_status();
 }
 
+// Row pitch (elements) of the transposed activations [K][M] the explicit
+// transpose writes: M rounded up to a multiple of 8, so every row is 16-byte
+// aligned for the gather's 16-byte copies.
+inline int64_t xt_pitch(int64_t M) { return (M + 7) / 8 * 8; }
+
 // Validation, the optional explicit transpose and the GEMM launch shared by
 // spgemm_tw_f16 (Y [M][N], y_nm false) and spgemm_tw_f16_yt (Y^T [N][M]).
 spg_status run(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc, void* Y, int64_t ldy, int64_t M,
@@ -702,7 +719,7 @@ spg_status run(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc
   if (!desc->offsetn || !desc->tile_n0 || !desc->tile_kofs || !desc->offsetk || !desc->Wc) return SPG_ERR_INVALID_ARG;
   if (x_layout == SPG_X_MK ? ldx < K : ldx < M) return SPG_ERR_INVALID_ARG;
   if (M == 0) return SPG_OK;  // empty batch: nothing is read or written
-  if (M % 8 || M >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
+  if (M >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(X, 16) || !aligned(Y, 2) || ldx % 8) return SPG_ERR_MISALIGNED;
   if (y_nm && (!aligned(Y, 16) || ldy % 8)) return SPG_ERR_MISALIGNED;
   if (x_layout == SPG_X_MK) {
@@ -717,11 +734,11 @@ spg_status run(const void* X, int64_t ldx, int x_layout, const spg_tw_desc* desc
   if (x_layout == SPG_X_MK) {
     uint16_t* ws = static_cast<uint16_t*>(workspace);
     dim3 grid(static_cast<unsigned>((K + 63) / 64), static_cast<unsigned>((M + 63) / 64));
+    ldt = xt_pitch(M);
     if (launch_pdl(transpose_kernel, grid, dim3(256), 0, s, static_cast<const uint16_t*>(X), ldx, int(M), int(K), ws,
-                   M) != cudaSuccess)
+                   ldt) != cudaSuccess)
       return SPG_ERR_CUDA;
     xt = ws;
-    ldt = M;
   }
   return launch_gemm(xt, ldt, desc, static_cast<uint16_t*>(Y), ldy, M, s, y_nm);
 }
@@ -768,7 +785,7 @@ spg_status tw_query_sizes(int64_t N, int64_t K, int32_t G, int64_t n_pruned, con
 
 size_t tw_workspace_size(int64_t M, int64_t K, int x_layout) {
   if (x_layout != SPG_X_MK || M <= 0 || K <= 0) return 0;
-  return static_cast<size_t>((M * K * 2 + 255) / 256 * 256);
+  return static_cast<size_t>((spg::tw::xt_pitch(M) * K * 2 + 255) / 256 * 256);
 }
 
 spg_status tw_reorganize(const void* W, int64_t ldw, int64_t n_pruned, const int32_t* k_per_tile,
@@ -839,8 +856,9 @@ spg_status spgemm_tw_f16_noalloc(const void* X, int64_t ldx, const spg_tw_desc* 
   if (M <= 0 || N <= 0 || K <= 0 || ldy < N || ldx < K) return SPG_ERR_INVALID_ARG;
   if (desc->G != kG || desc->T <= 0 || desc->offsetk_len <= 0 || desc->offsetk_len % kKBlock) return SPG_ERR_INVALID_ARG;
   if (!desc->offsetn || !desc->tile_n0 || !desc->tile_kofs || !desc->offsetk || !desc->Wc) return SPG_ERR_INVALID_ARG;
-  if (M % 8 || M >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
-  if (uint64_t(M) * uint64_t(K) * 2u > kNoAllocScratchBytes) return SPG_ERR_UNSUPPORTED_SHAPE;
+  if (M >= (int64_t(1) << 31)) return SPG_ERR_UNSUPPORTED_SHAPE;
+  const int64_t ldt = xt_pitch(M);
+  if (uint64_t(ldt) * uint64_t(K) * 2u > kNoAllocScratchBytes) return SPG_ERR_UNSUPPORTED_SHAPE;
   if (!aligned(X, 16) || !aligned(Y, 2) || ldx % 8) return SPG_ERR_MISALIGNED;
   spg_status st = check_device();
   if (st != SPG_OK) return st;
@@ -851,9 +869,9 @@ spg_status spgemm_tw_f16_noalloc(const void* X, int64_t ldx, const spg_tw_desc* 
   // so nothing left in the array by an earlier call is ever read
   dim3 tgrid(static_cast<unsigned>((K + 63) / 64), static_cast<unsigned>((M + 63) / 64));
   if (launch_pdl(transpose_kernel, tgrid, dim3(256), 0, s, static_cast<const uint16_t*>(X), ldx, int(M), int(K), xt,
-                 M) != cudaSuccess)
+                 ldt) != cudaSuccess)
     return SPG_ERR_CUDA;
-  return launch_gemm(xt, M, desc, static_cast<uint16_t*>(Y), ldy, M, s);
+  return launch_gemm(xt, ldt, desc, static_cast<uint16_t*>(Y), ldy, M, s);
 }
 
 }  // extern "C"

@@ -60,6 +60,9 @@ def test_host_only_calls():
     assert L.tw_query_sizes(768, 8256, 128, 77, kpt, ctypes.byref(sz)) == 2    # K above the reorganiser's limit
     assert L.tw_query_sizes(768, 768, 128, 77, None, ctypes.byref(sz)) == 1
     assert L.tw_workspace_size(4096, 768, spg.SPG_X_MK) == 4096 * 768 * 2
+    # a ragged M: the transposed rows are padded to a multiple of 8 elements
+    assert L.tw_workspace_size(15, 64, spg.SPG_X_MK) == (16 * 64 * 2 + 255) // 256 * 256
+    assert L.tw_workspace_size(129, 768, spg.SPG_X_MK) == (136 * 768 * 2 + 255) // 256 * 256
     assert L.tw_workspace_size(4096, 768, spg.SPG_X_KM) == 0
 
 
@@ -69,11 +72,13 @@ def test_validation_rejects_before_touching_the_device():
     L = spg.lib()
     assert L.spgemm_24_f16(None, 256, None, None, None, None, 256, 64, 256, 256, 0, None) == 1
     assert L.spgemm_24_f16(16, 100, 16, 16, None, 16, 256, 64, 256, 256, 0, None) == 1   # ldx < K
-    assert L.spgemm_24_f16(16, 256, 16, 16, None, 16, 256, 64, 256, 192, 0, None) == 2   # K % 128
+    assert L.spgemm_24_f16(16, 256, 16, 16, None, 16, 256, 64, 256, 160, 0, None) == 2   # K % 64
+    assert L.spgemm_24_f16(16, 256, 16, 16, None, 16, 256, 64, 256, 32, 0, None) == 2    # K < 64
     assert L.spgemm_24_f16(18, 256, 16, 16, None, 16, 256, 64, 256, 256, 0, None) == 3   # X misaligned
     assert L.spgemm_24_f16(16, 256, 16, 16, None, 16, 256, 64, 256, 256, 7, None) == 1   # dtype
     assert L.spgemm_24_s8(16, 256, 16, 16, None, None, 16, 256, 0, 64, 256, 256, None) == 1  # scale needed
-    assert L.spgemm_24_s8(16, 256, 16, 16, None, None, 16, 256, 1, 64, 256, 128, None) == 2  # K % 256
+    assert L.spgemm_24_s8(16, 256, 16, 16, None, None, 16, 256, 1, 64, 256, 192, None) == 2  # K % 128
+    assert L.spgemm_24_s8(16, 256, 16, 16, None, None, 16, 256, 1, 64, 256, 64, None) == 2   # K < 128
     assert L.sparse_prune_24(16, 6, 16, 6, 2, 6, 0, None) == 2                               # K % 4
     assert L.sparse_compress_24(16, 12, 16, 16, 2, 12, 0, None) == 2                         # K % 8
     assert L.sparse_prune_24(16, 8, 16, 8, 0, 8, 0, None) == 0                               # empty: no-op
@@ -133,7 +138,8 @@ def test_empty_batch_is_a_no_op():
                             None) == 0
     # zero-size torch tensors report a row stride of 1 ([N, 0] outputs, [K, 0] inputs): not checked
     assert L.spgemm_24_f16_yt(None, 256, Wv, meta, None, None, 1, 0, 256, 256, 0, None) == 0
-    assert L.spgemm_24_f16(None, 256, Wv, meta, None, None, 256, 0, 256, 192, 0, None) == 2   # K % 128
+    assert L.spgemm_24_f16(None, 256, Wv, meta, None, None, 256, 0, 256, 160, 0, None) == 2   # K % 64
+    assert L.spgemm_24_f16(None, 256, Wv, meta, None, None, 256, 0, 256, 192, 0, None) == 0   # K % 64 is enough
     assert L.spgemm_24_f16(None, 256, None, meta, None, None, 256, 0, 256, 256, 0, None) == 1  # no Wv
     assert L.spgemm_24_f16(None, 256, Wv, meta, None, None, 256, -1, 256, 256, 0, None) == 1  # M < 0
     assert L.spgemm_24_s8(None, 256, Wv, meta, None, None, None, 256, 0, 0, 256, 256, None) == 1  # scale

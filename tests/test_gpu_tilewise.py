@@ -1,7 +1,8 @@
 """GPU parity of the tile-wise path (reorganisation, transpose, gather GEMM) against the CPU oracle.
 
 The descriptor (offsetn, tile spans, offsetk, condensed values) must be
-bit-exact; the GEMM must match within |y - y_ref| <= 1e-3*sqrt(K) + 1e-2*|y_ref|
+bit-exact; the GEMM must match within max abs error 1e-3*sqrt(K) and max rel
+error 1e-2 (where |y_ref| exceeds the absolute bound)
 and be bit-exact when X is the identity (one product per output).
 """
 import numpy as np
@@ -59,7 +60,7 @@ def _check_desc(desc, ref):
 
 def _small_ties(seed, N=300, K=256, P=30):
     rng = np.random.default_rng(seed)
-    W = (rng.integers(-3, 4, (N, K)) * 0.25).astype(np.float16)   # many exact ties
+    W = (rng.integers(-3, 4, (N, K)) * (0.25 / 32)).astype(np.float16)   # many exact ties, weight-sized values
     T = (N - P + 127) // 128
     kpt = rng.integers(1, K + 1, T)
     kpt[0] = 1          # a tile keeping a single row
@@ -145,7 +146,7 @@ def test_wide_span_windows_and_pitch(spg, ldy_pad):
     import torch
     rng = np.random.default_rng(11)
     N, K, P, M = 640, 128, 320, 200
-    W = rng.standard_normal((N, K)).astype(np.float16)
+    W = (rng.standard_normal((N, K)) / 64).astype(np.float16)
     W[:P] = (W[:P].astype(np.float32) * 1e-3).astype(np.float16)   # the first P columns are pruned first
     kpt = rng.integers(1, K + 1, (N - P + 127) // 128)
     X = rng.standard_normal((M, K)).astype(np.float16)
@@ -176,7 +177,7 @@ def test_short_last_tile_aligned_pitch(spg, seed):
     import torch
     rng = np.random.default_rng(100 + seed)
     N, K, P, M = 264, 128, 5, 136
-    W = rng.standard_normal((N, K)).astype(np.float16)
+    W = (rng.standard_normal((N, K)) / 64).astype(np.float16)
     kpt = rng.integers(1, K + 1, (N - P + 127) // 128)
     X = rng.standard_normal((M, K)).astype(np.float16)
     desc = spg.tw_reorganize(torch.from_numpy(W).cuda(), 128, P, kpt)

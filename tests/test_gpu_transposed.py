@@ -63,7 +63,7 @@ def test_24_yt_is_the_transpose(spg, kind, M, N, K):
 
 def _tw_case(seed, N=300, K=256, P=30):
     rng = np.random.default_rng(seed)
-    W = (rng.integers(-3, 4, (N, K)) * 0.25).astype(np.float16)
+    W = (rng.integers(-3, 4, (N, K)) * (0.25 / 32)).astype(np.float16)
     T = (N - P + 127) // 128
     kpt = rng.integers(1, K + 1, T)
     return W, P, kpt
