@@ -81,3 +81,20 @@ def test_chain_fc1_gelu_quant_fc2_bit_exact(spg):
     acc2 = s24.gemm_24_s8_ref(H_ref, *s24.compress_24(fc2["W"], "s8"))
     Y_ref = s24.dequant_s8(acc2, fc2["scale"], fc2["bias"])
     assert np.array_equal(Y.cpu().numpy().view(np.uint16), Y_ref.view(np.uint16))
+
+
+def test_vitl_fc1_gelu_codes_within_one_of_plain_fp64_gelu(spg):
+    """The int8 codes of the fused GELU/quantise epilogue against the plain
+    definition in fp64: q = clamp(rne(GELU(v) * qscale), -127, 127) with
+    v = acc * scale[n] + bias[n] and GELU(v) = v * Phi(v) (scipy's erf).  The
+    epilogue works in fp32 with a published erf approximation (|error| <=
+    3e-7), so a code may differ by one where v * qscale sits next to a
+    rounding boundary, and by no more."""
+    d = gen.make_inputs("vitl_mlp_chain_s8", layers=["fc1"])[0]
+    got = _q_case(spg, d["X"], d["W"], d["scale"], d["bias"], d["qscale"], spg.SPG_ACT_GELU, pad=0)
+    acc = s24.gemm_24_s8_ref(d["X"], *s24.compress_24(d["W"], "s8")).astype(np.float64)
+    v = acc * d["scale"].astype(np.float64)[None, :] + d["bias"].astype(np.float64)[None, :]
+    want = np.clip(np.rint(s24.gelu_ref(v) * np.float64(d["qscale"])), -127, 127).astype(np.int64)
+    diff = np.abs(got.astype(np.int64) - want)
+    assert diff.max() <= 1
+    assert (diff == 0).mean() > 0.999          # off by one only next to a rounding boundary
