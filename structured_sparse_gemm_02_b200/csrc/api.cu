@@ -12,6 +12,8 @@
 namespace spg {
 
 __device__ uint32_t g_error_word;
+// The value spg_check_device_error() took out of g_error_word, for the host to read.
+__device__ uint32_t g_error_taken;
 
 namespace {
 constexpr int kMaxDevices = 64;
@@ -116,6 +118,11 @@ __global__ void selftest_wait_kernel(uint32_t* err, uint64_t limit_ns) {
   if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, err, ERR_WAIT_SELFTEST, limit_ns);
 }
 
+// Takes the error word and clears it in one atomic step, so a bit that a
+// kernel on another stream sets at the same moment is either taken now or
+// left for the next check, never lost.
+__global__ void take_error_word_kernel() { g_error_taken = atomicExch(&g_error_word, 0u); }
+
 }  // namespace spg
 
 extern "C" {
@@ -139,10 +146,12 @@ spg_status spg_check_device_error(spg_stream_t stream, uint32_t* bits) {
   if (bits) *bits = 0;
   spg_status st = spg::check_device();
   if (st != SPG_OK) return st;
-  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return SPG_ERR_CUDA;
-  uint32_t v = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&v, spg::g_error_word, sizeof(v)) != cudaSuccess) return SPG_ERR_CUDA;
-  if (v && cudaMemcpyToSymbol(spg::g_error_word, &zero, sizeof(zero)) != cudaSuccess) return SPG_ERR_CUDA;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  spg::take_error_word_kernel<<<1, 1, 0, s>>>();
+  if (cudaGetLastError() != cudaSuccess) return SPG_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SPG_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpyFromSymbol(&v, spg::g_error_taken, sizeof(v)) != cudaSuccess) return SPG_ERR_CUDA;
   if (bits) *bits = v;
   return v ? SPG_ERR_TIMEOUT : SPG_OK;
 }
