@@ -4,14 +4,18 @@
 ``python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]``
 
 One step is one pass of the workload's sparse layers over one batch of
-synthetic inputs already resident in HBM (default workload: the 2:4 fp16
-ViT-Base MLP, fc1 12608x3072x768 and fc2 12608x768x3072, each with its fused
-bias).  Prints ONE JSON line on rank 0.  Under torchrun every rank runs its
-own batch (weak scaling, no collective on the data path); the reported value
-is all ranks' dense-equivalent FLOPs divided by the slowest rank's time.
+synthetic inputs already resident in HBM (default workload: the largest
+configuration, the 2:4 bf16 prefill layer X[8192,4096] x W[16384,4096]^T).
+Prints ONE JSON line on rank 0.  Under torchrun every rank runs its own batch
+(weak scaling, no collective on the data path); the reported value is all
+ranks' dense-equivalent FLOPs divided by the slowest rank's time.  At one GPU
+the line also carries a ``configs`` block: every configuration (the tiny
+layer, the ViT-Base MLP, the int8 ViT-Large layer, the tile-wise BERT layers
+with [M, K] and [K, M] activations, the bf16 decode and prefill layers) timed
+per launch from graph replays, with its roofline fraction.
 
-``--impl reference`` times the CPU oracle (numpy, fp64) on the host cores on a
-bounded sample of the same workload instead.
+``--impl reference`` times the plain C++ oracle (fp64 / exact int64 sums, on
+all host cores) on a bounded sample of the same workload instead.
 """
 from __future__ import annotations
 
@@ -302,42 +306,173 @@ def tw_algorithmic(layers_tw, es=2):
     return flops, byts
 
 
-def run_ours(args, rank, world, local_rank):
-    import torch
-    import structured_sparse_gemm_02_b200 as spg
-    spg.lib()
-    torch.cuda.set_device(local_rank)
-    cfg = gen.CONFIGS[args.workload]
-    inputs = gen.make_inputs(args.workload, batch=rank)   # each rank its own activation batch
+def build_layers(spg, workload, rank, x_km=False, y_nm=False, gelu=False, min_copies=3):
+    """Device-resident layers of a workload with enough rotating buffer sets
+    that the sets one step cycles through exceed 3x the 126 MB L2.  Returns a
+    dict with the layers, the inputs, the kind, the copy count, the step's
+    bytes, and the algorithmic FLOPs and bytes of one step."""
+    cfg = gen.CONFIGS[workload]
+    inputs = gen.make_inputs(workload, batch=rank)   # each rank its own activation batch
     kind = cfg.kind
-    # rotating buffer sets: enough that the sets one step cycles through exceed 3x the 126 MB L2
     if kind in ("tw_f16", "tw_f32"):
         es = 4 if kind == "tw_f32" else 2
-        step_bytes = sum(es * (d["M"] * d["K"] * (2 if not args.x_km else 1) + d["M"] * d["N"]) for d in inputs)
+        step_bytes = sum(es * (d["M"] * d["K"] * (2 if not x_km else 1) + d["M"] * d["N"]) for d in inputs)
     else:
         step_bytes = sum(algorithmic_bytes(d, kind) for d in inputs)
-    copies = max(args.copies, int(math.ceil(3 * L2_BYTES / step_bytes)))
+    copies = max(min_copies, int(math.ceil(3 * L2_BYTES / step_bytes)))
     if kind == "tw_f16":
-        layers = [LayerTW(spg, d, copies, spg.SPG_X_KM if args.x_km else spg.SPG_X_MK, args.y_nm) for d in inputs]
+        layers = [LayerTW(spg, d, copies, spg.SPG_X_KM if x_km else spg.SPG_X_MK, y_nm) for d in inputs]
         flops_alg, bytes_alg = tw_algorithmic(layers)
     elif kind == "tw_f32":
-        if args.y_nm:
+        if y_nm:
             raise SystemExit("--y-nm applies to the fp16 tile-wise and 2:4 workloads")
-        layers = [LayerTW32(spg, d, copies, spg.SPG_X_KM if args.x_km else spg.SPG_X_MK) for d in inputs]
+        layers = [LayerTW32(spg, d, copies, spg.SPG_X_KM if x_km else spg.SPG_X_MK) for d in inputs]
         flops_alg, bytes_alg = tw_algorithmic(layers, es=4)
     else:
-        if args.y_nm and kind not in ("24_f16", "24_bf16"):
+        if y_nm and kind not in ("24_f16", "24_bf16"):
             raise SystemExit("--y-nm applies to the 16-bit 2:4 and tile-wise workloads")
-        if args.gelu and (kind not in ("24_f16", "24_bf16") or args.y_nm):
+        if gelu and (kind not in ("24_f16", "24_bf16") or y_nm):
             raise SystemExit("--gelu applies to the 16-bit 2:4 workloads with [M, N] outputs")
-        # --gelu: the activation of an MLP block, fused into its first layer
-        layers = [Layer24(spg, d, kind, copies, args.y_nm, args.gelu and j == 0) for j, d in enumerate(inputs)]
+        # gelu: the activation of an MLP block, fused into its first layer
+        layers = [Layer24(spg, d, kind, copies, y_nm, gelu and j == 0) for j, d in enumerate(inputs)]
         for j, L in enumerate(layers):
             if L.X is None:        # a chained layer reads the previous layer's output buffers
                 L.X = layers[j - 1].Y
         flops_alg = layer_flops(inputs) / 2.0
         bytes_alg = sum(algorithmic_bytes(d, kind) for d in inputs)
-    flops_dense = layer_flops(inputs)
+    return {"workload": workload, "cfg": cfg, "inputs": inputs, "kind": kind, "layers": layers, "copies": copies,
+            "step_bytes": step_bytes, "flops_alg": flops_alg, "bytes_alg": bytes_alg,
+            "flops_dense": layer_flops(inputs), "x_km": x_km}
+
+
+def capture_graph(fn, gstream):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=gstream):
+        fn()
+    return g
+
+
+def per_layer_times(W, reps, gstream, stream):
+    """Per-launch milliseconds of every layer: a graph of `copies` launches of
+    the layer over its rotating buffer sets, replayed `reps` times, timed with
+    events on the stream the replays run on."""
+    import torch
+    layers, copies = W["layers"], W["copies"]
+    graphs = [capture_graph(lambda L=L: [L.run(i) for i in range(copies)], gstream) for L in layers]
+    torch.cuda.synchronize()
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    out = []
+    for g in graphs:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        out.append(a.elapsed_time(b) / (reps * copies))
+    del graphs
+    return out
+
+
+def roofline(W, lay_ms, peaks, src):
+    """Roofline of the workload's dominant kernel: algorithmic work per launch
+    over the mean per-launch time, against the measured peak that bounds it."""
+    kind, nl = W["kind"], len(W["layers"])
+    inputs = W["inputs"]
+    mean_s = float(np.mean(lay_ms)) * 1e-3
+    if kind == "tw_f32":
+        # fp32 fused multiply-add on the CUDA cores: kept FLOPs per launch against the fp32 pipe
+        # peak, 148 SMs x 128 lanes x 2 FLOPs at the 1965 MHz maximum SM clock
+        peak = FP32_SMS * FP32_LANES * 2 * FP32_MAX_MHZ * 1e6 / 1e12
+        achieved = W["flops_alg"] / nl / mean_s / 1e12
+        return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": profiled_traffic(W["workload"]),
+                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
+                "scope": "whole library call per layer" + ("" if W["x_km"] else
+                                                           " (includes the [M, K] -> [K, M] transpose)"),
+                "kernel": "tw_gemm_f32_kernel"}
+    if kind == "tw_f16" or (kind == "24_bf16" and inputs[0]["M"] <= 64):
+        # HBM-bound shapes: algorithmic bytes per launch over the measured copy bandwidth
+        achieved = W["bytes_alg"] / nl / mean_s / 1e9
+        out = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+               "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic(W["workload"]),
+               "peak_source": f"{src} HBM copy bandwidth",
+               "kernel": "tw_gemm_kernel" if kind == "tw_f16" else "spgemm24_kernel"}
+        if kind == "tw_f16":
+            out["scope"] = "whole library call per layer" + ("" if W["x_km"] else
+                                                            " (includes the [M, K] -> [K, M] transpose)")
+        return out
+    # dense-equivalent FLOPs per launch against the 2:4 sparse tensor peak of the dtype:
+    # measured dense bf16 (same rate as fp16) x2 for 2:4 sparsity, x2 again for int8
+    ratio = 2.0 * (2.0 if kind == "24_s8" else 1.0)
+    peak = peaks["bf16_tflops"] * ratio
+    achieved = W["flops_dense"] / nl / mean_s / 1e12
+    return {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": achieved / peak, "traffic": profiled_traffic(W["workload"]),
+            "peak_source": f"{src} burst bf16 dense x{ratio:g} (2:4 sparse rate)",
+            "kernel": "spgemm24_kernel"}
+
+
+# The configurations timed in the `configs` block: (label, workload, x_km)
+CONFIG_BLOCK = [
+    ("tiny_f16", "tiny_f16", False),
+    ("vitb_mlp_f16", "vitb_mlp_f16", False),
+    ("vitl_mlp_s8", "vitl_mlp_s8", False),
+    ("tw_bert_f16 [M,K]", "tw_bert_f16", False),
+    ("tw_bert_f16 [K,M]", "tw_bert_f16", True),
+    ("bf16_decode", "bf16_decode", False),
+    ("bf16_prefill", "bf16_prefill", False),
+]
+
+
+def config_block(spg, peaks, src, gstream, stream, reps_target=200, skip=None):
+    """Every configuration's per-launch times (graph replays over rotating
+    buffer sets larger than 3x L2) and roofline fraction."""
+    import torch
+    out = []
+    for label, workload, x_km in CONFIG_BLOCK:
+        W = build_layers(spg, workload, 0, x_km=x_km)
+        copies = W["copies"]
+        # about 200 launches per layer, at least 3 replays of the graph
+        reps = max(3, reps_target // copies)
+        for L in W["layers"]:       # warm-up, eager
+            for i in range(copies):
+                L.run(i)
+        torch.cuda.synchronize()
+        lay_ms = per_layer_times(W, reps, gstream, stream)
+        if spg.check_device_error() != 0:
+            raise RuntimeError(f"device error word set while timing {label}")
+        step_s = sum(lay_ms) * 1e-3
+        ent = {"config": label, "note": W["cfg"].note,
+               "layers": [f"{d['layer']} {d['M']}x{d['N']}x{d['K']}" for d in W["inputs"]],
+               "per_layer_us": [1e3 * v for v in lay_ms],
+               "dense_eq_tflops": W["flops_dense"] / step_s / 1e12,
+               "effective_tflops": W["flops_alg"] / step_s / 1e12,
+               "l2": f"{copies} rotating sets of {W['step_bytes'] / 1e6:.1f} MB",
+               "launches_timed_per_layer": reps * copies}
+        if workload == "tiny_f16":
+            ent["roofline"] = {"bound": "latency", "note": "8.4 MFLOP per launch: launch latency, parity case"}
+        else:
+            r = roofline(W, lay_ms, peaks, src)
+            ent["roofline"] = {k: r[k] for k in ("bound", "achieved", "peak", "unit", "frac", "kernel")}
+        out.append(ent)
+        del W
+        torch.cuda.empty_cache()
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import structured_sparse_gemm_02_b200 as spg
+    spg.lib()
+    torch.cuda.set_device(local_rank)
+    W = build_layers(spg, args.workload, rank, x_km=args.x_km, y_nm=args.y_nm, gelu=args.gelu,
+                     min_copies=args.copies)
+    cfg, inputs, kind, layers, copies = W["cfg"], W["inputs"], W["kind"], W["layers"], W["copies"]
+    flops_alg, flops_dense, step_bytes = W["flops_alg"], W["flops_dense"], W["step_bytes"]
     stream = torch.cuda.current_stream()
     torch.cuda.synchronize()
 
@@ -360,21 +495,11 @@ def run_ours(args, rank, world, local_rank):
     nl = len(layers)
     gstream = torch.cuda.Stream()
     gstream.wait_stream(stream)
-
-    def capture(fn):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=gstream):
-            fn()
-        return g
-
-    g_full = capture(lambda: [step(i) for i in range(copies)])
+    g_full = capture_graph(lambda: [step(i) for i in range(copies)], gstream)
     rem = args.steps % copies
-    g_rem = capture(lambda: [step(i) for i in range(rem)]) if rem else None
-    g_layer = [capture(lambda L=L: [L.run(i) for i in range(copies)]) for L in layers]
+    g_rem = capture_graph(lambda: [step(i) for i in range(rem)], gstream) if rem else None
     torch.cuda.synchronize()
     g_full.replay()
-    for g in g_layer:
-        g.replay()
     torch.cuda.synchronize()
 
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -397,18 +522,10 @@ def run_ours(args, rank, world, local_rank):
     clocks = sampler.stop()
     total_ms = ev0.elapsed_time(ev1)
     reps = max(1, min(200, args.steps // copies))
-    per_layer = []
-    for g in g_layer:
-        a, b2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            g.replay()
-        b2.record(stream)
-        torch.cuda.synchronize()
-        per_layer.append([a.elapsed_time(b2) / (reps * copies)])
+    lay_ms = per_layer_times(W, reps, gstream, stream)
     if spg.check_device_error() != 0:
         raise RuntimeError("device error word set during the timed region")
-    del g_full, g_rem, g_layer
+    del g_full, g_rem
     dense = dense_baseline(layers, kind, copies, reps, gstream, stream, args) if args.dense_baseline else None
 
     total_ms = max_over_ranks(total_ms, world, "cuda")
@@ -422,36 +539,7 @@ def run_ours(args, rank, world, local_rank):
     e2e["value"] = aggregate_tflops(world, flops_dense, 1, e2e["ms_per_step"])
 
     peaks, src = load_peaks()
-    lay_ms = [float(np.mean(p)) for p in per_layer]
-    if kind == "tw_f32":
-        # fp32 fused multiply-add on the CUDA cores: kept FLOPs per launch against the fp32 pipe
-        # peak, 148 SMs x 128 lanes x 2 FLOPs at the 1965 MHz maximum SM clock
-        peak = FP32_SMS * FP32_LANES * 2 * FP32_MAX_MHZ * 1e6 / 1e12
-        achieved = flops_alg / nl / (np.mean(lay_ms) * 1e-3) / 1e12
-        roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
-                "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x 1965 MHz",
-                "scope": "whole library call per layer" + ("" if args.x_km else " (includes the [M, K] -> [K, M] transpose)"),
-                "kernel": "tw_gemm_f32_kernel"}
-    elif kind == "24_bf16" and inputs[0]["M"] <= 64 or kind == "tw_f16":
-        # HBM-bound shapes: algorithmic bytes per launch over the measured copy bandwidth
-        per_launch_bytes = bytes_alg / nl
-        achieved = per_launch_bytes / (np.mean(lay_ms) * 1e-3) / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": profiled_traffic(args.workload),
-                "peak_source": src,
-                "kernel": "tw_gemm_kernel" if kind == "tw_f16" else "spgemm24_kernel"}
-    else:
-        # dense-equivalent FLOPs per launch against the 2:4 sparse tensor peak of the dtype:
-        # measured dense bf16 (same rate as fp16) x2 for 2:4 sparsity, x2 again for int8
-        ratio = 2.0 * (2.0 if kind == "24_s8" else 1.0)
-        peak = peaks["bf16_tflops"] * ratio
-        per_launch = flops_dense / nl
-        achieved = per_launch / (np.mean(lay_ms) * 1e-3) / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": profiled_traffic(args.workload),
-                "peak_source": f"{src} burst bf16 dense x{ratio:g} (2:4 sparse rate)",
-                "kernel": "spgemm24_kernel"}
+    roof = roofline(W, lay_ms, peaks, src)
     out = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -471,6 +559,10 @@ def run_ours(args, rank, world, local_rank):
         "dense_cublas": dense,
         "clocks": clocks,
     }
+    del W, layers
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_configs:
+        out["configs"] = config_block(spg, peaks, src, gstream, stream)
     return out
 
 
@@ -571,9 +663,11 @@ def oracle_step(inputs, kind, rows_frac=1.0):
 
     2:4 layers: selection and compression, then the fp64 (fp16 / bf16) or exact
     int64 (int8, with the fp32 dequantisation) product over the masked weight.
-    Tile-wise layers: the numpy oracle's reorganisation (its exact integer
-    norms), then the C++ expansion to a dense weight and its fp64 product.
-    The int8 chain's GELU + quantisation step is the numpy oracle's."""
+    fp16 tile-wise layers: the C++ reorganisation (exact integer norms), its
+    expansion to a dense weight and the fp64 product.  fp32 tile-wise
+    layers: the pattern and the fp32 values through it from the numpy
+    oracle, then the C++ expansion and product.  The int8 chain's GELU +
+    quantisation step is the numpy oracle's."""
     from oracle import native, sparse24 as s24, tilewise as tw
     flops = 0.0
     prev = None
@@ -583,13 +677,15 @@ def oracle_step(inputs, kind, rows_frac=1.0):
         if rows_frac < 1.0:
             rows = np.arange(0, M, max(1, int(round(1.0 / rows_frac))))
             M = len(rows)
-        if kind in ("tw_f16", "tw_f32"):
-            r = tw.tw_reorganize(d["W16"] if kind == "tw_f32" else d["W"], d["G"], d["n_pruned"], d["k_per_tile"])
-            if kind == "tw_f32":
-                r = tw.tw_condense_values(d["W"], r)
+        if kind == "tw_f16":
+            kk = np.asarray(d["k_per_tile"], dtype=np.int32)
+            offsetn, kofs, offsetk, Wc = native.tw_reorganize(d["W"], d["n_pruned"], kk, d["G"])
+            Wd = native.tw_expand(d["N"], d["K"], offsetn, kofs, kk, offsetk, Wc)
+            native.gemm_f64(d["X"], Wd, rows=rows)
+        elif kind == "tw_f32":
+            r = tw.tw_condense_values(d["W"], tw.tw_reorganize(d["W16"], d["G"], d["n_pruned"], d["k_per_tile"]))
             offsetn, kofs, kk, offsetk, Wc = native.tw_descriptor(r)
-            if kind == "tw_f32":
-                Wc = np.ascontiguousarray(Wc.transpose(0, 2, 1))
+            Wc = np.ascontiguousarray(Wc.transpose(0, 2, 1))
             Wd = native.tw_expand(d["N"], d["K"], offsetn, kofs, kk, offsetk, Wc)
             native.gemm_f64(d["X"], Wd, rows=rows)
         elif kind == "24_s8":
@@ -635,7 +731,9 @@ def time_oracle(workload, budget_s):
     sample = (f"{reps} pass(es) of the oracle over "
               + ("all rows" if frac >= 1.0 else f"every {int(round(1 / frac))}th row")
               + f" of every layer of {workload} (plain C++ oracle: fp64 / exact int64 sequential sums,"
-              " OpenMP over rows; includes compression)")
+              " OpenMP over rows; includes compression"
+              + ("; the fp32 tile-wise pattern and values from the numpy oracle" if cfg.kind == "tw_f32" else "")
+              + ")")
     return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cpu_cores(), "kind": "oracle",
             "sample": sample, "seconds": dt}
 
@@ -662,7 +760,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="vitb_mlp_f16", choices=sorted(gen.CONFIGS))
+    ap.add_argument("--workload", default="bf16_prefill", choices=sorted(gen.CONFIGS))
     ap.add_argument("--copies", type=int, default=3)
     ap.add_argument("--x-km", action="store_true", help="tile-wise: activations already [K, M]")
     ap.add_argument("--y-nm", action="store_true",
@@ -673,6 +771,7 @@ def main():
                     help="also time dense cuBLAS GEMMs of the same shapes and report the speedup")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the per-configuration block")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
