@@ -287,3 +287,23 @@ def test_tw_all_zero_weight_rows_and_columns(spg):
     Y = _tw_run(spg, X, desc, 0, N, "y")
     rep = compare.check_close(Y.astype(np.float64), tw.tw_gemm_ref(X, ref), K)
     assert rep["ok"], rep
+
+
+@pytest.mark.parametrize("K", [832, 3072])
+def test_tw_long_k(spg, K):
+    """K above 768 (the BERT FFN output layer has K = 3072): the activation
+    slab of a row block no longer fits in shared memory, and the kept rows are
+    gathered from global memory instead.  Both layouts, a ragged M."""
+    import torch
+    rng = np.random.default_rng(K)
+    N, P, M = 300, 21, 203
+    W = (rng.standard_normal((N, K)) / 64).astype(np.float16)
+    kpt = rng.integers(1, K + 1, (N - P + 127) // 128)
+    desc = spg.tw_reorganize(torch.from_numpy(W).cuda(), 128, P, kpt)
+    ref = tw.tw_reorganize(W, 128, P, kpt)
+    X = rng.standard_normal((M, K)).astype(np.float16)
+    for layout in (0, 1):
+        for out in ("y", "yt"):
+            Y = _tw_run(spg, X, desc, layout, N, out)
+            rep = compare.check_close(Y.astype(np.float64), tw.tw_gemm_ref(X, ref), K)
+            assert rep["ok"], rep
