@@ -64,8 +64,26 @@ __host__ __device__ constexpr bool out_bf16(int k) { return k == OUT_BF16 || k =
 __host__ __device__ constexpr bool out_gelu(int k) { return k == OUT_F16_G || k == OUT_BF16_G || k == OUT_S8QG; }
 __host__ __device__ constexpr bool out_s8(int k) { return k == OUT_S8Q || k == OUT_S8QG; }
 
-// GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), in fp32.
-__device__ __forceinline__ float gelu_f32(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
+// GELU(v) = v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)), in fp32, for the 16-bit
+// epilogues (checked against the fp64 definition within the output tolerance).
+// erfc from Abramowitz & Stegun 7.1.26: for u >= 0,
+//   erfc(u) = (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-u^2),  t = 1 / (1 + p u),
+// with |error| <= 1.5e-7, evaluated branch-free with the hardware reciprocal
+// and base-2 exponential approximations:
+//   Phi(v) = 1 - erfc(|v| / sqrt 2) / 2 for v >= 0, erfc(|v| / sqrt 2) / 2 otherwise.
+__device__ __forceinline__ float gelu_f32(float v) {
+  const float u = fabsf(v) * 0.70710678118654752f;
+  float t, ex;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(t) : "f"(fmaf(0.3275911f, u, 1.0f)));
+  float poly = fmaf(t, 1.061405429f, -1.453152027f);
+  poly = fmaf(t, poly, 1.421413741f);
+  poly = fmaf(t, poly, -0.284496736f);
+  poly = fmaf(t, poly, 0.254829592f);
+  poly *= t;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ex) : "f"(-(u * u) * 1.4426950408889634f));  // exp(-u^2)
+  const float half_erfc = 0.5f * poly * ex;
+  return v * (v >= 0.0f ? 1.0f - half_erfc : half_erfc);
+}
 
 // GELU for the quantised path, where the rounded result decides an integer
 // code and must be reproducible bit for bit on the host: erf from

@@ -275,3 +275,40 @@ def test_gelu_epilogue_vitb_fc1_sampled(spg):
     ref = s24.gelu_ref(s24.gemm_24_ref(d["X"], *s24.compress_24(d["W"], "f16"), d["bias"], "f16", rows=rows))
     rep = compare.check_close(Y.cpu().numpy()[rows].astype(np.float64), ref, d["K"])
     assert rep["ok"], rep
+
+
+@pytest.mark.parametrize("kind", ["f16", "bf16"])
+def test_gelu_epilogue_sweep_identity_input(spg, kind):
+    """X = I: every output before the activation is one weight plus the bias,
+    exact in fp32, so the fused GELU is checked value by value over [-8, 8]
+    against fp64 GELU: within one unit in the last place of the output type
+    wherever the pre-activation is >= -2, and within the stated absolute bound
+    1e-3*sqrt(K) in the tail below.  (The epilogue's erfc approximation bounds
+    the absolute error, 1.5e-7; in the negative tail GELU falls below 0.05
+    and its relative error may grow, far inside the absolute bound.  The
+    outputs here reach +-8, where one bf16 rounding alone exceeds the absolute
+    bound of K = 256, so that bound is not applied to them.)"""
+    import torch
+    K, N = 256, 512
+    rng = np.random.default_rng(17)
+    cv = (lambda a: a.astype(np.float16)) if kind == "f16" else gen.f32_to_bf16_bits
+    W = cv(rng.uniform(-8.0, 8.0, (N, K)).astype(np.float32))
+    b = cv((rng.standard_normal(N) * 0.25).astype(np.float32))
+    X = cv(np.eye(K, dtype=np.float32))
+    Wd = to_dev(W, kind)
+    Wv, meta = spg.sparse_compress_24(Wd)
+    Y = spg.spgemm_24_f16_gelu(to_dev(X, kind), Wv, meta, to_dev(b, kind))
+    assert spg.check_device_error() == 0
+    got = s24.to_f64(to_host(Y.contiguous(), kind), kind)
+    pre = s24.to_f64(np.ascontiguousarray(s24.prune_24(W, kind).T), kind) + s24.to_f64(b, kind)[None, :]
+    ref = s24.gelu_ref(pre)
+    if kind == "f16":
+        ulp = np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64)
+        ulp = np.maximum(ulp, 2.0 ** -24)
+    else:
+        e = np.floor(np.log2(np.maximum(np.abs(ref), 2.0 ** -126)))
+        ulp = 2.0 ** (e - 7)
+    near = pre >= -2.0
+    assert np.all(np.abs(got - ref)[~near] <= compare.atol_for(K))
+    assert np.all(np.abs(got - ref)[near] <= ulp[near]), float(np.max((np.abs(got - ref) / ulp)[near]))
+    assert (pre < -3).any() and (pre > 3).any()
