@@ -146,6 +146,24 @@ spg_status spgemm_24_f16(const void* X, int64_t ldx, const void* Wv, const uint8
                          spg_stream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * spgemm_24_f16_host  [GPUSQ, Abstract; the layer called from host memory]
+ *
+ * spgemm_24_f16 on activations and outputs in HOST memory: X_host [M, K]
+ * (pitch ldx_host >= K elements) is copied into the caller's device buffer
+ * X_dev (pitch K), the layer writes Y_dev [M, N] (pitch ldy_dev), and Y_dev
+ * is copied to Y_host [M, N] (pitch ldy_host >= N), all asynchronously on
+ * `stream` (cudaMemcpy2DAsync; host memory should be page-locked for the
+ * copies to be asynchronous).  Nothing is allocated: X_dev needs M*K*2 bytes
+ * and Y_dev M*ldy_dev*2 bytes.  Wv, meta, bias and dtype as spgemm_24_f16;
+ * X_dev and Y_dev must satisfy its alignment rules (16-byte aligned, ldy_dev
+ * in bytes a multiple of 16).  The host buffers must stay valid until the
+ * stream reaches the copy-out.
+ * ------------------------------------------------------------------------- */
+spg_status spgemm_24_f16_host(const void* X_host, int64_t ldx_host, const void* Wv, const uint8_t* meta,
+                              const void* bias, void* Y_host, int64_t ldy_host, int64_t M, int64_t N, int64_t K,
+                              spg_dtype dtype, void* X_dev, void* Y_dev, int64_t ldy_dev, spg_stream_t stream);
+
+/* ---------------------------------------------------------------------------
  * spgemm_24_f16_gelu  [GPUSQ, Abstract: the 2:4 layers of a vision
  * transformer; the activation between the two layers of its MLP block]
  *

@@ -49,6 +49,8 @@ SIGNATURES = {
     "sparse_prune_24": (ctypes.c_int, [_p, _i64, _p, _i64, _i64, _i64, ctypes.c_int, _p]),
     "sparse_compress_24": (ctypes.c_int, [_p, _i64, _p, _p, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_f16": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
+    "spgemm_24_f16_host": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p, _p,
+                                          _i64, _p]),
     "spgemm_24_f16_gelu": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_f16_yt": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _i64, _i64, _i64, _i64, ctypes.c_int, _p]),
     "spgemm_24_s8": (ctypes.c_int, [_p, _i64, _p, _p, _p, _p, _p, _i64, ctypes.c_int, _i64, _i64, _i64, _p]),
@@ -228,6 +230,39 @@ def spgemm_24_f16(X, Wv, meta, bias=None, Y=None, stream=None):
         _ptr(X), X.stride(0), _ptr(Wv), _ptr(meta), _ptr(bias), _ptr(Y), Y.stride(0), M, N, K,
         _dtype_code(X), _stream(stream)))
     return Y
+
+
+def _host_arg(t, name: str, dtypes, shape) -> None:
+    """A host tensor whose pointer goes to a host <-> device copy: dtype, shape,
+    row-major with unit column stride, in CPU memory."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cpu":
+        raise ValueError(f"{name} must be in host memory (it is on {t.device})")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected one of {tuple(dtypes)}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dim() == 2 and t.numel() > 0 and t.shape[1] > 1 and t.stride(1) != 1:
+        raise ValueError(f"{name} must be row-major with unit column stride")
+
+
+def spgemm_24_f16_host(X_host, Wv, meta, bias, Y_host, X_dev, Y_dev, stream=None):
+    """spgemm_24_f16 from and to host memory (page-locked for asynchronous
+    copies): X_host [M, K] -> X_dev [M, K] (contiguous), the layer into Y_dev
+    [M, N], Y_dev -> Y_host [M, N], all queued on the stream."""
+    dts = _types("float16", "bfloat16")
+    _arg(X_dev, "X_dev", dts, contiguous=True)
+    M, K, N = _check_24(X_dev, Wv, meta, dts)
+    _host_arg(X_host, "X_host", (X_dev.dtype,), (M, K))
+    _host_arg(Y_host, "Y_host", (X_dev.dtype,), (M, N))
+    _arg(bias, "bias", (X_dev.dtype,), (N,), contiguous=True, optional=True)
+    _arg(Y_dev, "Y_dev", (X_dev.dtype,), (M, N))
+    _check("spgemm_24_f16_host", lib().spgemm_24_f16_host(
+        _ptr(X_host), X_host.stride(0), _ptr(Wv), _ptr(meta), _ptr(bias), _ptr(Y_host), Y_host.stride(0), M, N, K,
+        _dtype_code(X_dev), _ptr(X_dev), _ptr(Y_dev), Y_dev.stride(0), _stream(stream)))
+    return Y_host
 
 
 def spgemm_24_f16_gelu(X, Wv, meta, bias=None, Y=None, stream=None):

@@ -931,6 +931,33 @@ spg_status spgemm_24_f16(const void* X, int64_t ldx, const void* Wv, const uint8
   return dispatch<false, true, OUT_BF16>(X, ldx, Wv, meta, bias, nullptr, Y, ldy, M, N, K, s);
 }
 
+// The same layer from and to host memory: X copied in, the GEMM, Y copied out,
+// all on `stream`, through caller-provided device buffers.
+spg_status spgemm_24_f16_host(const void* X_host, int64_t ldx_host, const void* Wv, const uint8_t* meta,
+                              const void* bias, void* Y_host, int64_t ldy_host, int64_t M, int64_t N, int64_t K,
+                              spg_dtype dtype, void* X_dev, void* Y_dev, int64_t ldy_dev, spg_stream_t stream) {
+  using namespace spg;
+  if (M < 0 || N <= 0 || K <= 0 || ldx_host < K || ldy_host < N) return SPG_ERR_INVALID_ARG;
+  if (M != 0 && (!X_host || !Y_host)) return SPG_ERR_INVALID_ARG;
+  // the device layer's own checks (X_dev with pitch K, Y_dev with pitch ldy_dev)
+  spg_status st = gemm24::validate_common(X_dev, K, Wv, meta, Y_dev, ldy_dev, M, N, K, 2, 2, 64);
+  if (st != SPG_OK) return st;
+  if (dtype != SPG_F16 && dtype != SPG_BF16) return SPG_ERR_INVALID_ARG;
+  if (M == 0) return SPG_OK;
+  st = check_device();
+  if (st != SPG_OK) return st;
+  auto s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpy2DAsync(X_dev, size_t(K) * 2, X_host, size_t(ldx_host) * 2, size_t(K) * 2, size_t(M),
+                        cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return SPG_ERR_CUDA;
+  st = spgemm_24_f16(X_dev, K, Wv, meta, bias, Y_dev, ldy_dev, M, N, K, dtype, stream);
+  if (st != SPG_OK) return st;
+  if (cudaMemcpy2DAsync(Y_host, size_t(ldy_host) * 2, Y_dev, size_t(ldy_dev) * 2, size_t(N) * 2, size_t(M),
+                        cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    return SPG_ERR_CUDA;
+  return SPG_OK;
+}
+
 spg_status spgemm_24_f16_gelu(const void* X, int64_t ldx, const void* Wv, const uint8_t* meta, const void* bias,
                               void* Y, int64_t ldy, int64_t M, int64_t N, int64_t K, spg_dtype dtype,
                               spg_stream_t stream) {

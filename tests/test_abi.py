@@ -82,6 +82,12 @@ def test_validation_rejects_before_touching_the_device():
     assert L.sparse_prune_24(16, 6, 16, 6, 2, 6, 0, None) == 2                               # K % 4
     assert L.sparse_compress_24(16, 12, 16, 16, 2, 12, 0, None) == 2                         # K % 8
     assert L.sparse_prune_24(16, 8, 16, 8, 0, 8, 0, None) == 0                               # empty: no-op
+    # the host-buffer call: host pointers required for a non-empty batch, then the device layer's checks
+    assert L.spgemm_24_f16_host(None, 256, 16, 16, None, 16, 256, 64, 256, 256, 0, 16, 16, 256, None) == 1
+    assert L.spgemm_24_f16_host(16, 100, 16, 16, None, 16, 256, 64, 256, 256, 0, 16, 16, 256, None) == 1  # ldx_host
+    assert L.spgemm_24_f16_host(16, 256, 16, 16, None, 16, 256, 64, 256, 160, 0, 16, 16, 256, None) == 2  # K % 64
+    assert L.spgemm_24_f16_host(16, 256, 16, 16, None, 16, 256, 64, 256, 256, 0, 18, 16, 256, None) == 3  # X_dev
+    assert L.spgemm_24_f16_host(None, 256, 16, 16, None, None, 256, 0, 256, 256, 0, None, None, 256, None) == 0
     # transposed outputs: the pitch of Y^T covers M, not N
     assert L.spgemm_24_f16_yt(16, 256, 16, 16, None, 16, 32, 64, 256, 256, 0, None) == 1  # ldyt < M
     assert L.spgemm_24_f16_yt(16, 256, 16, 16, None, 16, 68, 68, 256, 256, 0, None) == 3  # ldyt*2 % 16
