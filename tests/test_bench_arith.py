@@ -48,3 +48,24 @@ def test_dense_equivalent_work():
     assert bench.layer_flops(fc) / 1e9 == pytest.approx(2 * 59.49, rel=1e-3)
     (M, N, K, _b), = _layers("bf16_prefill").values()
     assert bench.layer_flops([{"M": M, "N": N, "K": K}]) / 1e9 == pytest.approx(1099.5, rel=1e-3)
+
+
+def test_configs_block_covers_every_configuration():
+    """The per-configuration block of the bench line times the five
+    configurations of the workload set: the tiny layer, the ViT-Base MLP,
+    the int8 ViT-Large layer, the tile-wise BERT layers (both activation
+    layouts) and the bf16 prefill / decode pair."""
+    names = [w for _, w, _ in bench.CONFIG_BLOCK]
+    for want in ("tiny_f16", "vitb_mlp_f16", "vitl_mlp_s8", "tw_bert_f16", "bf16_prefill", "bf16_decode"):
+        assert want in names
+    assert {x for _, w, x in bench.CONFIG_BLOCK if w == "tw_bert_f16"} == {False, True}
+    assert set(names) <= set(gen.CONFIGS)
+
+
+def test_default_workload_is_the_largest_configuration():
+    import argparse, sys
+    flops = {n: sum(2.0 * M * N * K for (_, M, N, K, _) in c.layers) / len(c.layers) for n, c in gen.CONFIGS.items()}
+    largest = max(flops, key=flops.get)
+    assert largest == "bf16_prefill"
+    src = open(bench.__file__).read()
+    assert 'ap.add_argument("--workload", default="bf16_prefill"' in src
