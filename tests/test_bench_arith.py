@@ -63,7 +63,6 @@ def test_configs_block_covers_every_configuration():
 
 
 def test_default_workload_is_the_largest_configuration():
-    import argparse, sys
     flops = {n: sum(2.0 * M * N * K for (_, M, N, K, _) in c.layers) / len(c.layers) for n, c in gen.CONFIGS.items()}
     largest = max(flops, key=flops.get)
     assert largest == "bf16_prefill"

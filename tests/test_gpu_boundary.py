@@ -307,3 +307,49 @@ def test_tw_long_k(spg, K):
             Y = _tw_run(spg, X, desc, layout, N, out)
             rep = compare.check_close(Y.astype(np.float64), tw.tw_gemm_ref(X, ref), K)
             assert rep["ok"], rep
+
+
+# ---- the largest sizes the contract names ---------------------------------------------------
+
+def test_tw_largest_k(spg):
+    """K = 8192, the reorganiser's limit (its per-tile row norms live in shared
+    memory): descriptor bit-exact, product within the bounds."""
+    import torch
+    from tests.test_gpu_tilewise import _check_desc
+    rng = np.random.default_rng(8192)
+    N, K, P, M = 300, 8192, 40, 96
+    W = (rng.standard_normal((N, K)) / 64).astype(np.float16)
+    kpt = np.array([1, 8192, 3000], dtype=np.int32)[:(N - P + 127) // 128]
+    desc = spg.tw_reorganize(torch.from_numpy(W).cuda(), 128, P, kpt)
+    ref = tw.tw_reorganize(W, 128, P, kpt)
+    _check_desc(desc, ref)
+    X = rng.standard_normal((M, K)).astype(np.float16)
+    Y = _tw_run(spg, X, desc, 0, N, "y")
+    rep = compare.check_close(Y.astype(np.float64), tw.tw_gemm_ref(X, ref), K)
+    assert rep["ok"], rep
+
+
+def test_24_f16_long_k(spg):
+    """K = 32768: 256 pipeline stages per tile."""
+    rng = np.random.default_rng(32768)
+    M, N, K = 40, 300, 32768
+    X, W = rng.standard_normal((M, K)).astype(np.float16), (rng.standard_normal((N, K)) * 0.02).astype(np.float16)
+    got = _gemm16(spg, "f16", X, W, None)
+    rep = compare.check_close(s24.to_f64(got, "f16"), s24.gemm_24_ref(X, *s24.compress_24(W, "f16"), None, "f16"), K)
+    assert rep["ok"], rep
+
+
+def test_24_s8_long_k_exact(spg):
+    """K = 65536 with int8 values of magnitude 127: accumulators reach
+    K/2 * 127^2 = 528,506,880 (close to 2^29), still exact in int32 (the
+    contract's K <= 2^17 keeps |acc| < 2^31)."""
+    rng = np.random.default_rng(65536)
+    M, N, K = 16, 256, 65536
+    X = rng.choice(np.array([-127, 127], np.int8), size=(M, K))
+    W = rng.choice(np.array([-127, 127, 0, 1], np.int8), size=(N, K))
+    W[:8] = 127
+    X[:4] = 127
+    acc = s24.gemm_24_s8_ref(X, *s24.compress_24(W, "s8"))
+    assert np.abs(acc).max() == (K // 2) * 127 * 127
+    got = _s8(spg, X, W, None, None, spg.SPG_OUT_S32)
+    assert np.array_equal(got.astype(np.int64), acc)
