@@ -236,15 +236,17 @@ __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restri
 // Work unit (tile t, 128-row block of X): D[j][m] = sum_i Wc_t[j][i] * X[m][offsetk_t[i]]
 // on the dense tensor cores (A = condensed tile, K-major; B = gathered rows of
 // Xt, MN-major), then Y[m][offsetn[tG+j]] = D[j][m] and +0 in the tile's
-// pruned columns.  Persistent CTAs with warp roles (384 threads):
-//   warps 0-1  loads: warp 0 lane 0 issues the TMA of the condensed tile
-//              block; each lane of both warps gathers kept rows of Xt with
-//              16-byte cp.async (warp w takes rows 32w..32w+31 of a block).
+// pruned columns.  Persistent CTAs with warp roles (512 threads):
+//   warps 0-3  loads: warp 0 lane 0 issues the TMA of the condensed tile
+//              block; each lane of the four warps gathers kept rows of Xt
+//              with 16-byte cp.async (warp w takes rows 16w..16w+15 of a
+//              block; four warps keep about twice the bytes in flight of
+//              two).
 //              The 64 row indices of a block are read one block ahead, and
 //              the scalars of the next unit one unit ahead, so no copy waits
 //              on a dependent index load.
-//   warp 2     TMEM owner and MMA issuer (two accumulators)
-//   warps 4-11 drain, in two groups of four warps that each own 64 rows of
+//   warp 4     TMEM owner and MMA issuer (two accumulators)
+//   warps 8-15 drain, in two groups of four warps that each own 64 rows of
 //              the unit: tcgen05.ld of the accumulator (released at once).  The
 //              16-byte-aligned middle of the unit's output span
 //              [tile_n0[t], tile_n0[t+1]) is assembled in double-buffered
@@ -259,7 +261,11 @@ constexpr int B_BYTES = kKBlock * BN * 2;  // 16 KB: 64 gathered rows x 128 m, t
 constexpr int STAGES = 4;
 constexpr int EPI_GROUPS = 2;              // drain groups of 4 warps, each owning RG rows of a unit
 constexpr int RG = BN / EPI_GROUPS;        // 64
-constexpr int THREADS = 128 + 128 * EPI_GROUPS;
+constexpr int kGatherWarps = 4;            // warps 0-3
+constexpr int kRowsPerWarp = 64 / kGatherWarps;
+constexpr int kMmaWarp = 4;
+constexpr int kDrainWarp0 = 8;             // a multiple of 4: warp & 3 is the TMEM lane quadrant
+constexpr int THREADS = 32 * kDrainWarp0 + 128 * EPI_GROUPS;
 constexpr int WIN = 184;                   // output columns staged per window (a multiple of 8)
 constexpr int WIN_ELEMS = RG * WIN;        // one staging buffer: [64 rows] x WIN, box-blocked
 constexpr int OFF_STG = STAGES * (A_BYTES + B_BYTES);
@@ -269,7 +275,7 @@ constexpr int SMEM = OFF_BAR + (2 * STAGES + 5) * 8 + 16 + 1024;
 static_assert(SMEM <= 232448, "shared memory budget");
 static_assert(WIN % 8 == 0 && (WIN_ELEMS * 2) % 1024 == 0 && OFF_STG % 1024 == 0, "staging blocks stay aligned");
 constexpr uint32_t TMEM_COLS = 256;
-constexpr int kLoadLanes = 64;             // cp.async arrivals per stage (two gather warps)
+constexpr int kLoadLanes = 32 * kGatherWarps;  // cp.async arrivals per stage
 
 __device__ __forceinline__ void tail_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
   int never = 0;
@@ -329,7 +335,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       tma_prefetch_desc(&tmY8);
     }
   }
-  if (warp == 2) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_holder, TMEM_COLS);
     tmem_relinquish();
   }
@@ -340,11 +346,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   griddep_launch_dependents();
   griddep_wait();  // the previous kernel's writes (Xt, or readers of Y) are complete
 
-  if (warp < 2) {
+  if (warp < kGatherWarps) {
     // ---------------- loads ----------------
     uint32_t g = 0;
     bool ok = true;
-    const int rbase = 32 * warp;  // this warp's rows within a block
+    const int rbase = kRowsPerWarp * warp;  // this warp's rows within a block
+    const int rlane = lane % kRowsPerWarp;  // the row whose index this lane holds
     const int a = (lane >> 3) & 1, c = lane & 7, hl = lane >> 4;
     int u = blockIdx.x;
     // scalars of the current unit, and the first row indices of its block 0
@@ -353,7 +360,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int t = u / MB;
       kofs = tile_kofs[t];
       KB = (tile_kofs[t + 1] - kofs) / kKBlock;
-      nxt = offsetk[kofs + rbase + lane];
+      nxt = offsetk[kofs + rbase + rlane];
     }
     while (ok && u < units) {
       const int mb = (u % MB) * BN;
@@ -372,9 +379,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int kb = 0; kb < KB; ++kb, ++g) {
         const int cur = nxt;
         if (kb + 1 < KB)
-          nxt = offsetk[kofs + (kb + 1) * kKBlock + rbase + lane];
+          nxt = offsetk[kofs + (kb + 1) * kKBlock + rbase + rlane];
         else if (un < units)
-          nxt = offsetk[kofs_n + rbase + lane];
+          nxt = offsetk[kofs_n + rbase + rlane];
         const int s = g % STAGES;
         const uint32_t use = g / STAGES;
         if (use > 0 && !mbar_wait_warp(&empty[s], (use - 1) & 1, abort_flag, err, ERR_WAIT_EMPTY)) {
@@ -390,7 +397,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         // B: kept rows of Xt, 128 m each, as two MN-major 128-byte-swizzled
         // atoms of 64 m (16-byte chunk c of row r at chunk c ^ (r % 8))
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < kRowsPerWarp / 2; ++i) {
           const int rl = 2 * i + hl;
           const int r = rbase + rl;
           const int rk = __shfl_sync(0xffffffffu, cur, rl);
@@ -408,7 +415,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (uint32_t q = (g > uint32_t(STAGES) ? g - STAGES : 0u); q < g; ++q)
         tail_wait(&full[q % STAGES], (q / STAGES) & 1, err);
     __syncwarp();
-  } else if (warp == 2) {
+  } else if (warp == kMmaWarp) {
     // ---------------- MMA ----------------
     // kind::f16 dense, fp16 inputs, fp32 accumulate, A K-major, B MN-major, M=128, N=128.
     // One thread issues, with single-thread bounded waits.
@@ -449,13 +456,13 @@ __global__ void __launch_bounds__(THREADS, 1)
       tail_wait(mma_done, 0, err);
     }
     __syncwarp();
-  } else if (warp >= 4) {
+  } else if (warp >= kDrainWarp0) {
     // ---------------- drain and scatter ----------------
-    // Group eg (warps 4-7: eg 0, warps 8-11: eg 1) drains rows [64 eg, 64 eg + 64)
+    // Group eg (warps 8-11: eg 0, warps 12-15: eg 1) drains rows [64 eg, 64 eg + 64)
     // of every unit: TMEM columns b*BN + 64 eg .. +63 of the lanes of quadrant q.
     const int q = warp & 3;
-    const int eg = (warp - 4) >> 2;
-    const int gtid = threadIdx.x - 128 - 128 * eg;  // 0..127 within the group
+    const int eg = (warp - kDrainWarp0) >> 2;
+    const int gtid = threadIdx.x - 32 * kDrainWarp0 - 128 * eg;  // 0..127 within the group
     const uint32_t bar_win = 1 + eg, bar_vote = 3 + eg;
     uint16_t* stg0 = reinterpret_cast<uint16_t*>(smem + OFF_STG + eg * (2 * WIN_ELEMS * 2));
     uint16_t* edge = reinterpret_cast<uint16_t*>(smem + OFF_EDGE + eg * (RG * 16 * 2));  // [64 rows][16]
@@ -632,7 +639,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, TMEM_COLS);
   }
