@@ -621,6 +621,16 @@ def dense_baseline(layers, kind, copies, reps, gstream, stream, args):
     return {"per_layer_us": per_layer, "what": what}
 
 
+def e2e_row_chunks(M, chunks):
+    """Row ranges [m0, m1) of the end-to-end leg's pipelined host-buffer calls,
+    covering [0, M) in order: min(chunks, M // 256) ranges (at least one) of
+    ceil(M / n) rows, the last one shorter by the remainder, so that no call
+    is much smaller than 256 rows."""
+    n = max(1, min(chunks, M // 256))
+    rows = (M + n - 1) // n
+    return [(c * rows, min(M, (c + 1) * rows)) for c in range(n) if c * rows < M]
+
+
 def measure_e2e(spg, layers, kind, args, stream):
     import torch
     steps = max(3, min(args.e2e_steps, args.steps))
@@ -644,8 +654,8 @@ def measure_e2e(spg, layers, kind, args, stream):
     # call each, so the copy in of one chunk, the layer on another and the copy
     # out of a third overlap (the two copy directions and the SMs run at once).
     M0 = layers[0].d["M"]
-    nchunk = max(1, min(args.e2e_chunks, M0 // 256)) if host_call else 1
-    rows = (M0 + nchunk - 1) // nchunk
+    ranges = e2e_row_chunks(M0, args.e2e_chunks) if host_call else [(0, M0)]
+    nchunk = len(ranges)
     streams = [torch.cuda.Stream() for _ in range(3)] if nchunk > 1 else [stream]
 
     def once():
@@ -656,8 +666,7 @@ def measure_e2e(spg, layers, kind, args, stream):
                 return
             start = torch.cuda.Event()
             start.record(stream)
-            for c in range(nchunk):
-                m0, m1 = c * rows, min(M0, (c + 1) * rows)
+            for c, (m0, m1) in enumerate(ranges):
                 s = streams[c % len(streams)]
                 s.wait_event(start)
                 spg.spgemm_24_f16_host(hx[0][m0:m1], L.Wv[0], L.meta[0], L.bias[0], hy[0][m0:m1],

@@ -68,3 +68,20 @@ def test_default_workload_is_the_largest_configuration():
     assert largest == "bf16_prefill"
     src = open(bench.__file__).read()
     assert 'ap.add_argument("--workload", default="bf16_prefill"' in src
+
+
+@pytest.mark.parametrize("M,chunks", [(8192, 16), (8192, 8), (8192, 1), (16, 16), (255, 16), (256, 16),
+                                      (600, 16), (12608, 16), (6304, 7), (1000, 3)])
+def test_e2e_row_chunks_cover_the_batch(M, chunks):
+    """The end-to-end leg's row chunks are in order, contiguous, non-empty and
+    cover [0, M) exactly; there are min(chunks, M // 256) of them (at least
+    one), all but the last of ceil(M / n) >= 256 rows."""
+    r = bench.e2e_row_chunks(M, chunks)
+    n = max(1, min(chunks, M // 256))
+    assert len(r) == n
+    assert r[0][0] == 0 and r[-1][1] == M
+    assert all(a < b for a, b in r)
+    assert all(r[i][1] == r[i + 1][0] for i in range(n - 1))
+    assert all(b - a == -(-M // n) for a, b in r[:-1])
+    if n > 1:
+        assert -(-M // n) >= 256
