@@ -254,7 +254,8 @@ __global__ void __launch_bounds__(256) transpose_kernel(const uint16_t* __restri
 //              places its kept column), and leaves as a few 2-D TMA stores;
 //              the ragged ends (at most 7 columns a side) are assembled the
 //              same way in a [128][16] edge buffer and leave with one store
-//              instruction per two rows for both ends.
+//              instruction per two rows for both ends, from the three warps
+//              of the group that did not issue the TMA stores.
 constexpr int BN = 128;                   // X rows per work unit
 constexpr int A_BYTES = kG * kKBlock * 2;  // 16 KB
 constexpr int B_BYTES = kKBlock * BN * 2;  // 16 KB: 64 gathered rows x 128 m, two 64-wide atoms
@@ -627,13 +628,14 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       // ragged ends (16-byte rows only): one instruction covers both edge
       // sectors of two rows; lanes 0-7 / 16-23 the head chunk, lanes 8-15 /
-      // 24-31 the tail chunk, of rows r and r + 4
-      if (vec_ok && (n0 < a0 || a1 < n1)) {
+      // 24-31 the tail chunk, of rows r and r + 1.  The group's first warp
+      // has just issued the TMA stores, so the other three share the rows.
+      if (vec_ok && (n0 < a0 || a1 < n1) && q != 0) {
         const int l16 = lane & 15;
         const int col = l16 < 8 ? e1 + l16 : a1 + l16 - 8;
         const bool mine = l16 < 8 ? (col >= n0 && col < a0 && col < n1) : (col < n1);
         if (mine)
-          for (int row = q + 4 * (lane >> 4); row < rows; row += 8)
+          for (int row = 2 * (q - 1) + (lane >> 4); row < rows; row += 6)
             Y[int64_t(mb + row) * ldy + col] = edge[row * 16 + l16];
       }
     }
