@@ -1,4 +1,4 @@
-"""Pins of the pass criterion every fp16/bf16 parity verdict goes through.
+"""Pins of the pass criterion every fp16/bf16 parity result goes through.
 
 The stated bounds are a maximum absolute error of 1e-3*sqrt(K) and a maximum
 relative error of 1e-2.  These cases sit just inside and just outside each
