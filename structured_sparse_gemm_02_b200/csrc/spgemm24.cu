@@ -635,6 +635,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       const bool full_n = nb + 32 <= N;
       const bool pair_full = n0 + 64 * (q >> 1) + 64 <= N;
       const uint32_t tbase = tmem + (uint32_t(32 * q) << 16) + uint32_t(b * BN);
+      constexpr bool kPaired = C::OUT_ES == 2 && !C::YT && !out_gelu(OUT);
+      if (kPaired && pair_full && sub < C::NCH) {
+        // 16-bit Y, whole pair box: two chunks per round, so one pair of
+        // barriers, one proxy fence and one store issue serve both
+#pragma unroll 1
+        for (int c = sub; c < C::NCH; c += 2 * kStride) {
+          const int c2 = c + kStride;
+          const bool two = c2 < C::NCH;
+          uint32_t h[32], h2[32];
+          tmem_ld_32x32b_x32(tbase + 32 * c, h);
+          if (two) tmem_ld_32x32b_x32(tbase + 32 * c2, h2);
+          tmem_ld_wait(h);
+          if (two) tmem_ld_wait(h2);
+          if ((two ? c2 : c) + kStride >= C::NCH) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(acc_empty_l + 8u * b);
+          }
+          const int mb = m0 + 32 * c, mb2 = m0 + 32 * c2;
+          if (mb >= M) continue;
+          const bool do2 = two && mb2 < M;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) h[j] = convert_pair16<OUT, kInt8>(h[2 * j], h[2 * j + 1], badd, sc, has_bias);
+          if (do2) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              h2[j] = convert_pair16<OUT, kInt8>(h2[2 * j], h2[2 * j + 1], badd, sc, has_bias);
+          }
+          const uint32_t boxa = pbox0 + (nst & 1) * 4096, boxb = pbox0 + ((nst + 1) & 1) * 4096;
+          if (nst >= 1) {
+            if (pair_lead && lane == 0) bulk_wait_read<0>();
+            named_bar_sync(pair_bar, 64);
+          }
+          stage_pair_box16(boxa, reinterpret_cast<const uint32_t(&)[16]>(h), lane, q & 1);
+          if (do2) stage_pair_box16(boxb, reinterpret_cast<const uint32_t(&)[16]>(h2), lane, q & 1);
+          fence_proxy_async_smem();
+          named_bar_sync(pair_bar, 64);
+          if (pair_lead && lane == 0) {
+            // one bulk group per box, so a single-chunk round that follows
+            // (bulk_wait_read<1>) sees the box it reuses finished
+            tma_store_2d_saddr(&tmY, boxa, n0 + 64 * (q >> 1), mb);
+            bulk_commit();
+            if (do2) {
+              tma_store_2d_saddr(&tmY, boxb, n0 + 64 * (q >> 1), mb2);
+              bulk_commit();
+            }
+          }
+          __syncwarp();
+          nst += do2 ? 2 : 1;
+        }
+      } else
 #pragma unroll 1
       for (int c = sub; c < C::NCH; c += kStride) {
         uint32_t h[32];
