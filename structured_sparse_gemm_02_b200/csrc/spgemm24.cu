@@ -635,10 +635,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       const bool full_n = nb + 32 <= N;
       const bool pair_full = n0 + 64 * (q >> 1) + 64 <= N;
       const uint32_t tbase = tmem + (uint32_t(32 * q) << 16) + uint32_t(b * BN);
-      constexpr bool kPaired = C::OUT_ES == 2 && !C::YT && !out_gelu(OUT);
+      constexpr bool kPaired = C::OUT_ES == 2 && !C::YT;
       if (kPaired && pair_full && sub < C::NCH) {
-        // 16-bit Y, whole pair box: two chunks per round, so one pair of
-        // barriers, one proxy fence and one store issue serve both
+        // 16-bit Y (with or without GELU), whole pair box: two chunks per
+        // round, so one pair of barriers, one proxy fence and one store issue
+        // serve both
 #pragma unroll 1
         for (int c = sub; c < C::NCH; c += 2 * kStride) {
           const int c2 = c + kStride;
